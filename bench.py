@@ -1,0 +1,436 @@
+"""Benchmark: fused W4A16 decode GEMV, HBM GB/s at M=1, K=4096, N=14336.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl wq|reference]
+
+One step = one fused dequant-in-register matmul Y[1, 14336] = X[1, 4096] *
+What^T over a Llama-8B gate/up-shaped INT4 layer (asymmetric, group 128,
+binary16 scale and zero), inputs resident in HBM.  Successive steps read
+different copies of the quantized layer from a pool larger than 4x the L2,
+so every step streams its weights from HBM.  Steps are replayed from CUDA
+graphs and timed with CUDA events on the launching stream.
+
+value       = algorithmic bytes of all steps on all GPUs / device time (GB/s)
+roofline    = the same per launch against the measured HBM copy bandwidth
+e2e         = the same metric through the Python API with X on the host
+              (pinned), copied in, and Y read back to the host every step
+cpu_baseline= the CPU oracle (plain C, float64) on the same layer
+
+For N > 1 (torchrun) each rank runs an independent replica on its own GPU
+(the decode GEMV has no exchange step); time is the max over ranks.
+``--impl reference`` times the CPU oracle as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W4A16 fused GEMV HBM GB/s (fraction of B200 peak) at M=1, K=4096, N=14336"
+M, K, N = 1, 4096, 14336
+BITS, GROUP, SYM = 4, 128, False
+WORKLOAD = ("decode GEMV, Llama-8B gate/up layer: M=1, K=4096, N=14336, INT4 asymmetric "
+            "group 128, fp16 scale+zero, bf16 X, fp32 Y")
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "gemv_w4a16_m1_k4096_n14336.json")
+KERNEL_SOURCES = [os.path.join(ROOT, "w4a16_decode_matmul_b200", "csrc", f)
+                  for f in ("gemv.cuh", "common.cuh")]
+
+
+def algorithmic_bytes(m: int = M, n: int = N, k: int = K, bits: int = BITS,
+                      group: int = GROUP, sym: bool = SYM, y_bytes: int = 4) -> int:
+    """Bytes the method must move per step: packed codes + scales (+ zeros)
+    + X + Y (page 1 section 2: N_param * b / 8 + metadata)."""
+    meta = n * (k // group) * 2 * (1 if sym else 2)
+    return n * k * bits // 8 + meta + m * k * 2 + m * n * y_bytes
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+# ----------------------------------------------------------------- ranks
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def reduce_max(value: float, device=None) -> float:
+    """Max of a float over all ranks (identity when not distributed)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(bytes_per_step: int, steps: int, world: int, max_ms: float) -> float:
+    """Aggregate throughput: every rank moves bytes_per_step per step."""
+    return bytes_per_step * steps * world / (max_ms * 1e-3) / 1e9
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                r = [x.strip() for x in r]
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+                for name, flag in zip(names, r[5:9]):
+                    if flag.lower() == "active":
+                        reasons.add(name)
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        top = sorted(sm)[len(sm) // 4:]        # samples taken under load
+        return {"sm_mhz": statistics.median(top), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- CPU oracle
+
+def oracle_threads() -> int:
+    return len(os.sched_getaffinity(0))
+
+
+def time_oracle(target_s: float, seed_w: int = 0, seed_x: int = 1):
+    """Time the oracle's matmul (decode from codes + float64 dot products) on
+    the same layer for about target_s seconds.  Returns (GB/s, steps, s)."""
+    os.environ.setdefault("OMP_NUM_THREADS", str(oracle_threads()))
+    import oracle
+    import synth
+    W = synth.weight(N, K, seed=seed_w)
+    X = synth.activation(M, K, seed=seed_x)
+    orc = oracle.get()
+    _, codes, scales, zeros = orc.quantize(synth.half_bits(W), BITS, GROUP, SYM)
+    xb = synth.bf16_bits(X)
+    steps, t0 = 0, time.perf_counter()
+    while True:
+        orc.matmul(xb, codes, scales, zeros, N, K, BITS, GROUP, SYM)
+        steps += 1
+        el = time.perf_counter() - t0
+        if el >= target_s:
+            break
+    return algorithmic_bytes() * steps / el / 1e9, steps, el
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    warm = max(1, min(args.warmup, 2))
+    time_oracle(0.0)  # builds + warms the oracle
+    for _ in range(warm - 1):
+        time_oracle(0.0)
+    target = max(5.0, min(30.0, 0.05 * args.steps))
+    gbs, steps, el = time_oracle(target)
+    cores = int(os.environ.get("OMP_NUM_THREADS", oracle_threads()))
+    sample = (f"oracle matmul over the full {K}x{N} layer at M=1, {steps} steps in "
+              f"{el:.1f} s (bounded sample of the benchmark's step count)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": steps, "warmup": warm, "ms_per_step": el / steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": WORKLOAD, "M": M, "K": K, "N": N,
+                                        "bits": BITS, "group": GROUP, "symmetric": SYM},
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------- GPU arm
+
+def run_wq(args):
+    import torch
+    import torch.distributed as dist
+
+    rank, world, local = dist_env()
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    import synth
+    import w4a16_decode_matmul_b200 as wq
+
+    # one quantized layer, replicated into a pool larger than 4x L2
+    W = synth.weight(N, K, seed=0).to(dev)
+    base = wq.quantize(W, bits=BITS, group=GROUP, symmetric=SYM)
+    del W
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    layer_bytes = base.nbytes
+    pool_n = max(2, -(-4 * l2 // layer_bytes) + 1)
+    pool = [wq.QuantizedWeight(base.codes.clone(), base.scales.clone(),
+                               None if base.zeros is None else base.zeros.clone(),
+                               N, K, BITS, GROUP, SYM) for _ in range(pool_n)]
+    X = synth.activation(M, K, seed=1).to(dev)
+    Y = torch.empty(M, N, dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(dev)
+
+    def capture(count: int):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            wq.matmul(X, pool[0], out=Y)        # warm the binding on this stream
+            stream.synchronize()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(count):
+                    wq.matmul(X, pool[i % pool_n], out=Y)
+        return g
+
+    steps = args.steps
+    full, rest = divmod(steps, pool_n)
+    g_full = capture(pool_n)
+    g_rest = capture(rest) if rest else None
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, -(-max(args.warmup, 3) // pool_n))):
+            g_full.replay()
+    stream.synchronize()
+
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(f"GPU-{torch.cuda.get_device_properties(dev).uuid}") as clocks:
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for _ in range(full):
+                g_full.replay()
+            if g_rest is not None:
+                g_rest.replay()
+            end.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    ms_local = start.elapsed_time(end)
+    ms = reduce_max(ms_local, dev)
+    clk = clocks.summary()
+    err = wq.get_device_error(dev)
+
+    bytes_step = algorithmic_bytes()
+    value = whole_job_gbs(bytes_step, steps, world, ms)
+    per_launch_ms = ms_local / steps
+    achieved = bytes_step / (per_launch_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_peaks()
+    traffic = None
+    if os.path.exists(PROFILE_SUMMARY):
+        prof = json.load(open(PROFILE_SUMMARY))
+        if prof.get("kernel_source_hash") == kernel_source_hash():
+            traffic = prof.get("dram_bytes_per_launch")
+
+    # comparison points on the same GPU (not part of the timed region)
+    extra = compare_points(wq, torch, dev, stream, pool, X, pool_n)
+
+    # end to end through the public API: host X in, host Y out, every step
+    e2e = measure_e2e(wq, torch, dev, pool, pool_n, args)
+
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
+        "steps": steps, "warmup": max(args.warmup, 3), "ms_per_step": ms / steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": M, "K": K, "N": N, "bits": BITS,
+                   "group": GROUP, "symmetric": SYM, "parallelism": f"replicas{world}",
+                   "l2": (f"rotating pool of {pool_n} weight copies "
+                          f"({pool_n * layer_bytes / 1e6:.0f} MB, "
+                          f"{pool_n * layer_bytes / l2:.1f}x the {l2 / 1e6:.0f} MB L2)"),
+                   "timing": f"CUDA graphs of {pool_n} launches, CUDA events on the launch stream"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": traffic, "peak_kind": f"{peak_kind} HBM copy"},
+        "us_per_layer": round(per_launch_ms * 1e3, 3),
+        "frac_of_nominal_8tbs": round(achieved / 8000.0, 4),
+        "gpu_launches": steps,
+        "clocks": clk,
+        "e2e": e2e,
+        "device_status": err,
+        **extra,
+    }
+    if world == 1:
+        gbs, st, el = time_oracle(10.0)
+        line["cpu_baseline"] = {
+            "value": round(gbs, 4), "unit": "GB/s",
+            "cores": int(os.environ.get("OMP_NUM_THREADS", oracle_threads())),
+            "kind": "oracle",
+            "sample": f"oracle matmul over the full {K}x{N} layer at M=1, {st} steps in {el:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        del g_full, g_rest
+        dist.destroy_process_group()
+    return 0
+
+
+def compare_points(wq, torch, dev, stream, pool, X, pool_n, reps: int = 50):
+    """Dense bf16 GEMV (torch) and the unfused dequantize + GEMV on the same
+    shape, with the same rotation over copies; microseconds per layer."""
+    Wd = [torch.randn(N, K, device=dev, dtype=torch.bfloat16) for _ in range(
+        max(2, -(-4 * torch.cuda.get_device_properties(dev).L2_cache_size // (N * K * 2)) + 1))]
+    Wq_tmp = torch.empty(N, K, device=dev, dtype=torch.bfloat16)
+    Y = torch.empty(M, N, device=dev, dtype=torch.bfloat16)
+    Yf = torch.empty(M, N, device=dev, dtype=torch.float32)
+
+    def timed(fn, n):
+        with torch.cuda.stream(stream):
+            for i in range(3):
+                fn(i)
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record(stream)
+            for i in range(n):
+                fn(i)
+            e.record(stream)
+        torch.cuda.synchronize(dev)
+        return s.elapsed_time(e) / n * 1e3
+
+    dense_us = timed(lambda i: torch.matmul(X, Wd[i % len(Wd)].T, out=Y), reps)
+    unfused_us = timed(lambda i: (wq.dequantize(pool[i % pool_n], out=Wq_tmp),
+                                  torch.matmul(X, Wq_tmp.T, out=Y)), reps)
+    fused_us = timed(lambda i: wq.matmul(X, pool[i % pool_n], out=Yf), reps)
+    dense_bytes = N * K * 2 + M * K * 2 + M * N * 2
+    return {
+        "dense_bf16_gemv": {"us_per_layer": round(dense_us, 3),
+                            "gbs": round(dense_bytes / dense_us / 1e3, 1),
+                            "how": "torch.matmul bf16 [1,4096]x[4096,14336], eager"},
+        "unfused_dequant_then_gemv": {"us_per_layer": round(unfused_us, 3)},
+        "fused_eager_us_per_layer": round(fused_us, 3),
+        "fused_vs_dense_speedup": round(dense_us / fused_us, 3),
+    }
+
+
+def measure_e2e(wq, torch, dev, pool, pool_n, args):
+    """Public API with host buffers: pinned X copied in, Y read back, every
+    step, inside the timed region."""
+    import synth
+    Xh = synth.activation(M, K, seed=1).pin_memory()
+    Yh = torch.empty(M, N, dtype=torch.float32).pin_memory()
+    steps = max(50, min(2000, args.steps // 100))
+    for i in range(5):
+        wq.matmul(Xh, pool[i % pool_n], out=Yh)
+        torch.cuda.current_stream(dev).synchronize()
+    t0 = time.perf_counter()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record()
+    for i in range(steps):
+        wq.matmul(Xh, pool[i % pool_n], out=Yh)
+        torch.cuda.current_stream(dev).synchronize()     # the host reads Y
+    e.record()
+    torch.cuda.synchronize(dev)
+    wall = time.perf_counter() - t0
+    ms = reduce_max(max(s.elapsed_time(e), wall * 1e3), dev)
+    _, world, _ = dist_env()
+    return {"value": round(whole_job_gbs(algorithmic_bytes(), steps, world, ms), 3),
+            "unit": "GB/s", "h2d_bytes_per_step": M * K * 2,
+            "d2h_bytes_per_step": M * N * 4, "steps": steps,
+            "us_per_step": round(ms / steps * 1e3, 3)}
+
+
+def ncu_case():
+    """A small, self-contained launch sequence for ncu captures: one
+    quantize of the benchmark layer, then 8 fused matmuls on it."""
+    import torch
+    import synth
+    import w4a16_decode_matmul_b200 as wq
+    dev = torch.device("cuda", 0)
+    qw = wq.quantize(synth.weight(N, K, seed=0).to(dev), bits=BITS, group=GROUP, symmetric=SYM)
+    X = synth.activation(M, K, seed=1).to(dev)
+    Y = torch.empty(M, N, dtype=torch.float32, device=dev)
+    for _ in range(8):
+        wq.matmul(X, qw, out=Y)
+    torch.cuda.synchronize(dev)
+    assert wq.get_device_error(dev) == 0
+    print("ncu case ok")
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200000)
+    ap.add_argument("--warmup", type=int, default=2000)
+    ap.add_argument("--impl", choices=["wq", "reference"], default="wq")
+    ap.add_argument("--ncu-case", action="store_true",
+                    help="no timing: quantize the layer and run 8 fused matmuls, for ncu")
+    args = ap.parse_args(argv)
+    if args.ncu_case:
+        return ncu_case()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_wq(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,136 @@
+/*
+ * wq.h -- C ABI of the B200 (sm_100a) library for groupwise affine low-bit
+ * weight quantization and the fused dequant-in-register W4A16 matmul.
+ *
+ * Operations and where they are defined:
+ *   quantize    q = clamp(round(w/s) + z, qmin, qmax), one binary16 scale s
+ *               and one binary16 integer zero z per group of `group`
+ *               consecutive weights along K.  Asymmetric: "vLLM 量化与推测解码"
+ *               section 1 (affine map, min-max scale s = (xmax - xmin)/(qmax
+ *               - qmin), zero z = round(qmin - xmin/s), qmin = 0, qmax =
+ *               2^b - 1, range widened to contain 0, scale 1.0 for a
+ *               degenerate range, zero clamped).  Symmetric: "量化"
+ *               (llminference s08) section 解法 (z = 0, s = max|w| /
+ *               (2^(b-1) - 1), codes clipped to [-2^(b-1), 2^(b-1) - 1]).
+ *   dequantize  x^ = s (q - z)  (same section 1); materialises the weights.
+ *   matmul      Y = X * What^T with What = s (q - z) formed on chip
+ *               ("vLLM 量化与推测解码" section 2, W4A16: packed INT4 weights
+ *               and group scales are unpacked and scaled in registers /
+ *               on-chip tiles, multiplied with 16-bit activations and
+ *               accumulated in higher precision; "量化" (llminference s08)
+ *               section 实现: dequantize inside the accumulation, never write
+ *               full-precision weights back to memory).
+ *
+ * Numerics (fixed where the pages leave them open):
+ *   - round() is round-half-to-even; the arithmetic that decides each code
+ *     is exact for binary16 inputs;
+ *   - the stored scale is the binary16 value obtained by rounding the scale
+ *     toward +infinity, and codes are computed with that stored scale, so
+ *     |w - x^| <= s/2 holds for every element;
+ *   - the zero point is stored as a binary16 holding an integer;
+ *   - symmetric codes are stored offset-binary: u = q + 2^(b-1);
+ *   - matmul accumulates in binary32; |y - y_ref| <= 1e-4 * sum_k |x_k w^_k|
+ *     (binary32 output), plus one bfloat16 ulp for bfloat16 output.
+ *
+ * Layouts (all row-major, all device memory, all owned by the caller):
+ *   W      [N][K]              binary16 weights (quantize input)
+ *   codes  [N][K*bits/8]       bytes; bits = 4: byte j of a row holds
+ *                              k = 2j in bits 0-3 and k = 2j + 1 in bits 4-7;
+ *                              bits = 8: one byte per weight
+ *   scales [N][K/group]        binary16
+ *   zeros  [N][K/group]        binary16 (integers 0..2^b-1); asymmetric only,
+ *                              NULL when symmetric
+ *   X      [M][K]              bfloat16 activations
+ *   Y      [M][N]              binary32 or bfloat16 (fully overwritten)
+ *   What   [N][K]              bfloat16 (dequantize output)
+ *
+ * Ownership and streams: the caller allocates and frees every buffer.  No
+ * entry point allocates, frees or synchronizes; all work is enqueued on
+ * `stream` (a cudaStream_t; NULL is the legacy default stream).  Every
+ * pointer must be 16-byte aligned.  Inputs and outputs must not overlap.
+ *
+ * Errors: arguments are checked on the host before anything is launched; a
+ * failed check returns a non-zero status and launches nothing.  A launch
+ * failure returns WQ_ERR_CUDA.  Kernels never trap: a wait that exceeds its
+ * time limit records WQ_ERR_TIMEOUT in a device status word that
+ * wq_get_device_error() reads.  Weights containing NaN or Inf give
+ * unspecified codes.
+ */
+#ifndef WQ_H
+#define WQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st *wq_stream_t;
+
+typedef enum wq_status {
+    WQ_OK = 0,
+    WQ_ERR_INVALID_ARG = 1,  /* a size, pointer or option is out of range   */
+    WQ_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement */
+    WQ_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned            */
+    WQ_ERR_CUDA = 4,         /* a CUDA runtime call failed                  */
+    WQ_ERR_TIMEOUT = 5       /* a device-side wait ran out of time          */
+} wq_status;
+
+/* Output element types for wq_matmul. */
+enum { WQ_OUT_F32 = 0, WQ_OUT_BF16 = 1 };
+
+/* Supported formats: bits in {4, 8}; group in {32, 64, 128}; K a multiple of
+ * 32 and of group; 1 <= N, K < 2^31; 1 <= M. */
+
+/* Bytes of the packed codes of an [N][K] matrix: N*K*bits/8 ("vLLM 量化与推测
+ * 解码" section 2, payload N_param * b_w / 8).  Returns 0 for invalid sizes. */
+size_t wq_codes_bytes(int64_t N, int64_t K, int bits);
+
+/* Elements of each metadata tensor (scales, and zeros when asymmetric):
+ * N*(K/group).  Each element is 2 bytes.  Returns 0 for invalid sizes. */
+size_t wq_meta_elems(int64_t N, int64_t K, int group);
+
+/* Quantize W [N][K] binary16 into codes / scales / zeros (layouts above).
+ * symmetric = 0: asymmetric, zeros required; symmetric = 1: zeros must be
+ * NULL.  One pass over W; the result is bit-exact with the definition in
+ * the file header. */
+wq_status wq_quantize(const void *W, int64_t N, int64_t K, int bits, int group,
+                      int symmetric, void *codes, void *scales, void *zeros,
+                      wq_stream_t stream);
+
+/* Materialise What [N][K] bfloat16 = round-to-nearest-even(s (q - z)).
+ * Kept only as the traffic baseline of the unfused path (dequantize, then an
+ * ordinary matmul), which moves more bytes than the 16-bit weights it
+ * replaces ("量化" (llminference s08) section 实现). */
+wq_status wq_dequantize(const void *codes, const void *scales, const void *zeros,
+                        int64_t N, int64_t K, int bits, int group, int symmetric,
+                        void *W_out, wq_stream_t stream);
+
+/* Y [M][N] = X [M][K] * What^T, weights formed on chip from codes, scales
+ * and zeros and never written to memory.  out_dtype is WQ_OUT_F32 or
+ * WQ_OUT_BF16 (round-to-nearest-even from the binary32 accumulator).
+ * M <= 32 runs the small-batch decode kernel (codes streamed once from HBM,
+ * tensor-core products of integer-valued bfloat16 codes, binary32 group
+ * scaling); larger M runs the prefill kernel.  Deterministic: the same
+ * inputs give the same bits on every call. */
+wq_status wq_matmul(const void *X, int64_t M, const void *codes, const void *scales,
+                    const void *zeros, int64_t N, int64_t K, int bits, int group,
+                    int symmetric, void *Y, int out_dtype, wq_stream_t stream);
+
+/* Read and clear the device status word (WQ_OK if no kernel recorded an
+ * error).  Synchronizes `stream` first. */
+wq_status wq_get_device_error(wq_stream_t stream);
+
+/* Static text for a status code. */
+const char *wq_status_string(wq_status status);
+
+/* Library version string. */
+const char *wq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WQ_H */

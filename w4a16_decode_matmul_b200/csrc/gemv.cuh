@@ -1,0 +1,517 @@
+// gemv.cuh -- fused dequant-in-register small-batch matmul Y = X * What^T
+// (M <= 32): "vLLM 量化与推测解码" section 2 (W4A16: packed INT4 weights and
+// group scales are unpacked and scaled on chip, multiplied with 16-bit
+// activations, accumulated in higher precision; the full-precision weights
+// are never materialised) and "量化" (llminference s08) section 实现 (each
+// group's block is dequantized inside the accumulation).
+//
+// Decode is bound by the bytes of the packed weights ("量化" section 问题:
+// time = bytes / bandwidth), so the kernel is built around streaming the
+// codes exactly once at HBM speed with as few instructions per weight as
+// possible:
+//
+//   * Persistent CTAs, one per SM.  Work item = RT row tiles of 16 rows; the
+//     CTA's K range (all of K, or 1/C of it when a cluster of C CTAs splits
+//     K) is cut into stages.  One producer warp streams 16-row x 64-byte
+//     boxes of codes with TMA into a ring of DEPTH stages (mbarrier
+//     full/empty pairs), together with the stage's [16 rows x groups] scale
+//     and zero tiles, so tens of KB per SM are in flight regardless of
+//     register pressure.
+//   * 16 consumer warps.  Warp (rt, sk) owns row tile rt and BPW boxes of
+//     every stage.  Lane (g, t) of a warp holds rows g and g+8 and one
+//     quarter of every group, so each tensor-core step stays inside one group.
+//   * Unpacking: one LOP3 turns two 4-bit codes u into the bfloat16 pair
+//     (128 + u) (exponent 2^7, code in the low mantissa bits: exact); 8-bit
+//     codes go through a binary32 exponent trick and a paired conversion.
+//     The integer-valued operands enter mma.sync m16n8k16 (weights as the
+//     16-row A operand, activations as the 8-column B operand, binary32
+//     accumulation), which replaces 8 scalar FMAs per lane and step.
+//   * Per group, in binary32: y += s * (C - (128 + z) * Sx), where C is the
+//     group's tensor-core sum of x * (128 + u) and Sx the group's sum of x
+//     (precomputed once per CTA).  For 8-bit codes the bias is z.
+//   * The activations are staged in shared memory once per CTA, permuted so
+//     that every B fragment is one 8-byte load.
+//   * Deterministic reductions: warps of a row tile add their partial sums
+//     through shared memory in a fixed order; cluster ranks add theirs
+//     through distributed shared memory in rank order.
+#pragma once
+
+#include "common.cuh"
+
+namespace wq {
+namespace gemv {
+
+constexpr int kNumConsumerWarps = 16;
+constexpr int kThreads = (kNumConsumerWarps + 1) * 32;
+constexpr int kBoxRows = 16;
+constexpr int kBoxRowBytes = 64;
+constexpr int kBoxBytes = kBoxRows * kBoxRowBytes;  // 1 KB
+
+struct Params {
+  const __nv_bfloat16* X;  // [M][K]
+  void* Y;                 // [M][N]
+  const __half* scales;    // [N][ngroups] (used by the plain-load metadata path)
+  const __half* zeros;     // [N][ngroups] or null
+  int M, N, K, ngroups;
+  int row_tiles;           // ceil(N / 16)
+  int items;               // ceil(row_tiles / RT)
+  int RT, SKW, BPW;        // row tiles per item, warps per row tile, boxes per warp per stage
+  int depth;               // ring stages
+  int kc;                  // K extent of one cluster rank (multiple of max(box k, G))
+  int stage_k;             // SKW * BPW * box_k
+  int stages_per_item;     // ceil(kc / stage_k)
+  int meta_tma;            // 1: metadata tiles by TMA; 0: loaded by the producer warp
+  int y_bf16;
+  uint32_t stage_bytes;    // codes + metadata of one stage
+  uint32_t meta_offset;    // offset of the metadata inside a stage
+  uint32_t off_ring, off_x, off_sx, off_red, off_part;
+};
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4],
+                                               const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t bits) {
+  uint32_t r;
+  // (a & mask) | bits
+  asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(r) : "r"(a), "r"(mask), "r"(bits));
+  return r;
+}
+
+// Eight 4-bit codes of one 32-bit word -> four bfloat16 pairs (128 + u):
+// r[i] = (u_i, u_{i+4}) for i = 0..3 (low half first).
+__device__ __forceinline__ void unpack_u4(uint32_t w, uint32_t (&r)[4]) {
+  constexpr uint32_t kMask = 0x000F000Fu, kMagic = 0x43004300u;  // bf16 128.0 pair
+  r[0] = lop3_and_or(w, kMask, kMagic);
+  r[1] = lop3_and_or(w >> 4, kMask, kMagic);
+  r[2] = lop3_and_or(w >> 8, kMask, kMagic);
+  r[3] = lop3_and_or(w >> 12, kMask, kMagic);
+}
+
+// Four 8-bit codes -> two bfloat16 pairs (u0, u1), (u2, u3), exact integers.
+__device__ __forceinline__ void unpack_u8(uint32_t w, uint32_t (&r)[2]) {
+  float f[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    // 2^23 + u as binary32, minus 2^23: exact
+    f[i] = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7650 | i)) - 8388608.0f;
+  }
+  __nv_bfloat162 p0 = __floats2bfloat162_rn(f[0], f[1]);
+  __nv_bfloat162 p1 = __floats2bfloat162_rn(f[2], f[3]);
+  r[0] = *reinterpret_cast<uint32_t*>(&p0);
+  r[1] = *reinterpret_cast<uint32_t*>(&p1);
+}
+
+// Load N consecutive 32-bit words (N = 1, 2, 4) from shared memory.
+template <int N>
+__device__ __forceinline__ void load_words(uint32_t addr, uint32_t (&w)[N]) {
+  if constexpr (N == 4) {
+    const uint4 v = lds128(addr);
+    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+  } else if constexpr (N == 2) {
+    const uint2 v = lds64(addr);
+    w[0] = v.x; w[1] = v.y;
+  } else {
+    w[0] = lds32(addr);
+  }
+}
+
+template <int BITS, int G>
+struct Geometry {
+  static constexpr int kBoxK = kBoxRowBytes * 8 / BITS;           // k per box row
+  static constexpr int kGroupBytes = G * BITS / 8;                 // bytes of one group row
+  static constexpr int kU = kGroupBytes < kBoxRowBytes ? kGroupBytes : kBoxRowBytes;
+  static constexpr int kUk = kU * 8 / BITS;                        // k per sub-unit
+  static constexpr int kQB = kU / 4;                               // bytes per lane quarter
+  static constexpr int kQk = kUk / 4;                              // k per lane quarter
+  static constexpr int kWords = kQB / 4;                           // 32-bit words per quarter
+  static constexpr int kSubUnits = kBoxRowBytes / kU;              // sub-units per box
+  static constexpr int kStepsPerSubUnit = kUk / 16;
+  static constexpr int kSubUnitsPerGroup = G / kUk;                // 1, or 2 (8-bit, G = 128)
+  static_assert(kQB == 4 || kQB == 8 || kQB == 16, "quarter size");
+  static_assert(kQk % 8 == 0, "activation staging works in blocks of 8");
+};
+
+template <int BITS, bool SYM, int G, int MT>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemv_kernel(const __grid_constant__ CUtensorMap tmap_codes,
+                const __grid_constant__ CUtensorMap tmap_scales,
+                const __grid_constant__ CUtensorMap tmap_zeros, const Params p) {
+  using Geo = Geometry<BITS, G>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* empty = full + 32;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 512);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // Cluster geometry: rank splits K; cluster id walks the items.
+  const uint32_t rank = cluster_ctarank();
+  uint32_t csize;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(csize));
+  const int cid = int(cluster_id_x());
+  const int ncl = int(num_clusters_x());
+  const int k_begin = int(rank) * p.kc;
+  const int k_end = min(p.K, k_begin + p.kc);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < p.depth; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kNumConsumerWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  grid_dependency_wait();
+
+  uint8_t* ring = smem + p.off_ring;
+  constexpr bool kAsymMeta = !SYM;
+
+  if (warp == kNumConsumerWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmap_codes);
+      if (p.meta_tma) {
+        prefetch_tensormap(&tmap_scales);
+        if (kAsymMeta) prefetch_tensormap(&tmap_zeros);
+      }
+    }
+    const uint64_t policy = l2_policy_evict_first();
+    const uint32_t meta_rt_bytes = uint32_t(kBoxRows * (p.stage_k / G) * 2);
+    int slot = 0;
+    uint32_t phase = 0;
+    for (int item = cid; item < p.items; item += ncl) {
+      for (int st = 0; st < p.stages_per_item; ++st) {
+        if (!*abort_flag && !mbar_wait(&empty[slot], phase ^ 1)) *abort_flag = 1;
+        uint8_t* stage = ring + size_t(slot) * p.stage_bytes;
+        uint8_t* meta = stage + p.meta_offset;
+        const int stage_k0 = k_begin + st * p.stage_k;
+        const int g0 = stage_k0 / G;
+        // bytes this stage will receive by TMA
+        uint32_t bytes = 0;
+        for (int rt = 0; rt < p.RT; ++rt) {
+          const int tile = item * p.RT + rt;
+          if (tile >= p.row_tiles) continue;
+          for (int b = 0; b < p.SKW * p.BPW; ++b)
+            if (stage_k0 + b * Geo::kBoxK < k_end) bytes += kBoxBytes;
+          if (p.meta_tma) bytes += meta_rt_bytes * (kAsymMeta ? 2 : 1);
+        }
+        if (!p.meta_tma) {
+          // plain loads of the stage's metadata by the whole warp
+          const int sg = p.stage_k / G;
+          for (int rt = 0; rt < p.RT; ++rt) {
+            const int tile = item * p.RT + rt;
+            if (tile >= p.row_tiles) continue;
+            __half* ms = reinterpret_cast<__half*>(meta + rt * meta_rt_bytes);
+            __half* mz = reinterpret_cast<__half*>(meta + (p.RT + rt) * meta_rt_bytes);
+            for (int e = lane; e < kBoxRows * sg; e += 32) {
+              const int r = e / sg, gl = e % sg;
+              const int row = tile * kBoxRows + r, gi = g0 + gl;
+              const bool ok = row < p.N && gi < p.ngroups;
+              ms[e] = ok ? p.scales[size_t(row) * p.ngroups + gi] : __float2half(0.f);
+              if (kAsymMeta) mz[e] = ok ? p.zeros[size_t(row) * p.ngroups + gi] : __float2half(0.f);
+            }
+          }
+          __syncwarp();
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[slot], bytes);
+          if (!*abort_flag) {
+            for (int rt = 0; rt < p.RT; ++rt) {
+              const int tile = item * p.RT + rt;
+              if (tile >= p.row_tiles) continue;
+              const int row0 = tile * kBoxRows;
+              for (int sk = 0; sk < p.SKW; ++sk)
+                for (int bb = 0; bb < p.BPW; ++bb) {
+                  const int b = sk * p.BPW + bb;
+                  const int kb = stage_k0 + b * Geo::kBoxK;
+                  if (kb >= k_end) continue;
+                  tma_load_2d(stage + size_t((rt * p.SKW + sk) * p.BPW + bb) * kBoxBytes,
+                              &tmap_codes, &full[slot], kb * BITS / 8, row0, policy);
+                }
+              if (p.meta_tma) {
+                tma_load_2d(meta + rt * meta_rt_bytes, &tmap_scales, &full[slot], g0, row0,
+                            policy);
+                if (kAsymMeta)
+                  tma_load_2d(meta + (p.RT + rt) * meta_rt_bytes, &tmap_zeros, &full[slot], g0,
+                              row0, policy);
+              }
+            }
+          }
+        }
+        __syncwarp();
+        if (++slot == p.depth) {
+          slot = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    // Drain: every issued stage must have landed before the CTA may exit.
+    if (*abort_flag && lane == 0) {
+      for (int i = 0; i < p.depth; ++i) {
+        int s2 = slot - 1 - i;
+        uint32_t ph = phase;
+        if (s2 < 0) {
+          s2 += p.depth;
+          ph ^= 1;
+        }
+        mbar_wait(&full[s2], ph);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ consumers
+    const int tid = threadIdx.x;  // 0 .. 16*32-1
+    const int nthr = kNumConsumerWarps * 32;
+    const int M = p.M;
+    __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(smem + p.off_x);
+    float* sx = reinterpret_cast<float*>(smem + p.off_sx);
+    constexpr int kSxCols = 8 * MT;
+
+    // Stage X (permuted so that each B fragment is one 8-byte load) and the
+    // per-group sums of X for this rank's K range.
+    {
+      const int nblk = (k_end - k_begin) / 8;
+      for (int idx = tid; idx < M * nblk; idx += nthr) {
+        const int m = idx / nblk, kb = idx % nblk;
+        const int r = kb * 8;
+        const uint4 v = *reinterpret_cast<const uint4*>(p.X + size_t(m) * p.K + k_begin + r);
+        const int su = r / Geo::kUk, rr = r % Geo::kUk;
+        const int tq = rr / Geo::kQk, rq = rr % Geo::kQk;
+        uint2 c0, c1;
+        int slot0;
+        if (BITS == 4) {
+          slot0 = su * Geo::kStepsPerSubUnit + 2 * (rq / 8);
+          c0 = make_uint2(__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632));
+          c1 = make_uint2(__byte_perm(v.y, v.w, 0x5410), __byte_perm(v.y, v.w, 0x7632));
+        } else {
+          slot0 = su * Geo::kStepsPerSubUnit + rq / 4;
+          c0 = make_uint2(v.x, v.y);
+          c1 = make_uint2(v.z, v.w);
+        }
+        *reinterpret_cast<uint2*>(xs + (size_t(slot0) * M + m) * 16 + tq * 4) = c0;
+        *reinterpret_cast<uint2*>(xs + (size_t(slot0 + 1) * M + m) * 16 + tq * 4) = c1;
+      }
+      const int ng_local = (k_end - k_begin) / G;
+      for (int pr = warp; pr < ng_local * kSxCols; pr += kNumConsumerWarps) {
+        const int gl = pr / kSxCols, m = pr % kSxCols;
+        float acc = 0.f;
+        if (m < M) {
+          const __nv_bfloat16* xr = p.X + size_t(m) * p.K + k_begin + gl * G;
+#pragma unroll
+          for (int i = 0; i < G / 32; ++i) acc += __bfloat162float(xr[lane + 32 * i]);
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        }
+        if (lane == 0) sx[gl * kSxCols + m] = acc;
+      }
+    }
+    named_barrier_sync(1, nthr);
+
+    const int rt = warp / p.SKW, sk = warp % p.SKW;
+    const int g = lane >> 2, t = lane & 3;
+    const uint32_t xs_addr = smem_addr(xs);
+    const uint32_t sx_addr = smem_addr(sx);
+    float* red = reinterpret_cast<float*>(smem + p.off_red);
+    float* part = reinterpret_cast<float*>(smem + p.off_part);
+    const uint32_t meta_rt_bytes = uint32_t(kBoxRows * (p.stage_k / G) * 2);
+    const int sg = p.stage_k / G;
+
+    int slot = 0;
+    uint32_t phase = 0;
+    int local_item = 0;
+    for (int item = cid; item < p.items; item += ncl, ++local_item) {
+      const int tile = item * p.RT + rt;
+      const bool tile_ok = tile < p.row_tiles;
+      float y[MT][4];
+#pragma unroll
+      for (int nt = 0; nt < MT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) y[nt][e] = 0.f;
+      float c[2][MT][4];
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int nt = 0; nt < MT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) c[h][nt][e] = 0.f;
+
+      for (int st = 0; st < p.stages_per_item; ++st) {
+        if (!*abort_flag && !mbar_wait(&full[slot], phase)) *abort_flag = 1;
+        const uint8_t* stage = ring + size_t(slot) * p.stage_bytes;
+        const uint32_t stage_addr = smem_addr(stage);
+        const int stage_k0 = k_begin + st * p.stage_k;
+        const int g0 = stage_k0 / G;
+        const uint32_t meta_s = stage_addr + p.meta_offset + rt * meta_rt_bytes;
+        const uint32_t meta_z = stage_addr + p.meta_offset + (p.RT + rt) * meta_rt_bytes;
+        if (tile_ok && !*abort_flag) {
+          for (int bb = 0; bb < p.BPW; ++bb) {
+            const int b = sk * p.BPW + bb;
+            const int kb = stage_k0 + b * Geo::kBoxK;
+            if (kb >= k_end) break;
+            const uint32_t box = stage_addr + uint32_t((rt * p.SKW + sk) * p.BPW + bb) * kBoxBytes;
+#pragma unroll
+            for (int j = 0; j < Geo::kSubUnits; ++j) {
+              const int ksu = kb + j * Geo::kUk;
+              if (ksu >= k_end) break;
+              // codes of rows g and g+8, this lane's quarter of the sub-unit
+              uint32_t wa[Geo::kWords], wb[Geo::kWords];
+              const uint32_t ra = box + g * kBoxRowBytes + j * Geo::kU + t * Geo::kQB;
+              load_words<Geo::kWords>(ra, wa);
+              load_words<Geo::kWords>(ra + 8 * kBoxRowBytes, wb);
+              const int slot_base = (ksu - k_begin) / 16;
+#pragma unroll
+              for (int wi = 0; wi < Geo::kWords; ++wi) {
+                if (BITS == 4) {
+                  uint32_t ua[4], ub[4];
+                  unpack_u4(wa[wi], ua);
+                  unpack_u4(wb[wi], ub);
+#pragma unroll
+                  for (int h = 0; h < 2; ++h) {
+                    const uint32_t a[4] = {ua[2 * h], ub[2 * h], ua[2 * h + 1], ub[2 * h + 1]};
+                    const int sl = slot_base + 2 * wi + h;
+#pragma unroll
+                    for (int nt = 0; nt < MT; ++nt) {
+                      const int m = g + 8 * nt;
+                      uint32_t bf[2] = {0u, 0u};
+                      if (m < M) {
+                        const uint2 v = lds64(xs_addr + ((uint32_t(sl) * M + m) * 16 + t * 4) * 2);
+                        bf[0] = v.x;
+                        bf[1] = v.y;
+                      }
+                      mma_bf16_16816(c[h][nt], a, bf);
+                    }
+                  }
+                } else {
+                  uint32_t ua[2], ub[2];
+                  unpack_u8(wa[wi], ua);
+                  unpack_u8(wb[wi], ub);
+                  const uint32_t a[4] = {ua[0], ub[0], ua[1], ub[1]};
+                  const int sl = slot_base + wi;
+#pragma unroll
+                  for (int nt = 0; nt < MT; ++nt) {
+                    const int m = g + 8 * nt;
+                    uint32_t bf[2] = {0u, 0u};
+                    if (m < M) {
+                      const uint2 v = lds64(xs_addr + ((uint32_t(sl) * M + m) * 16 + t * 4) * 2);
+                      bf[0] = v.x;
+                      bf[1] = v.y;
+                    }
+                    mma_bf16_16816(c[wi & 1][nt], a, bf);
+                  }
+                }
+              }
+              // group epilogue: y += s * (C - bias * Sx)
+              if (((ksu + Geo::kUk) % G) == 0) {
+                const int gi = (ksu + Geo::kUk) / G - 1;
+                const int gls = gi - g0;
+                const int glx = gi - k_begin / G;
+                const uint32_t e0 = uint32_t(g * sg + gls) * 2;
+                const uint32_t e1 = uint32_t((g + 8) * sg + gls) * 2;
+                const float s0 = lds_half_as_float(meta_s + e0);
+                const float s1 = lds_half_as_float(meta_s + e1);
+                const float z0 = SYM ? float(1 << (BITS - 1)) : lds_half_as_float(meta_z + e0);
+                const float z1 = SYM ? float(1 << (BITS - 1)) : lds_half_as_float(meta_z + e1);
+                const float bias0 = (BITS == 4 ? 128.f : 0.f) + z0;
+                const float bias1 = (BITS == 4 ? 128.f : 0.f) + z1;
+#pragma unroll
+                for (int nt = 0; nt < MT; ++nt) {
+                  const uint2 sv = lds64(sx_addr + (glx * kSxCols + 8 * nt + 2 * t) * 4);
+                  const float sx0 = __uint_as_float(sv.x), sx1 = __uint_as_float(sv.y);
+                  const float d0 = c[0][nt][0] + c[1][nt][0];
+                  const float d1 = c[0][nt][1] + c[1][nt][1];
+                  const float d2 = c[0][nt][2] + c[1][nt][2];
+                  const float d3 = c[0][nt][3] + c[1][nt][3];
+                  y[nt][0] = fmaf(s0, fmaf(-bias0, sx0, d0), y[nt][0]);
+                  y[nt][1] = fmaf(s0, fmaf(-bias0, sx1, d1), y[nt][1]);
+                  y[nt][2] = fmaf(s1, fmaf(-bias1, sx0, d2), y[nt][2]);
+                  y[nt][3] = fmaf(s1, fmaf(-bias1, sx1, d3), y[nt][3]);
+#pragma unroll
+                  for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) c[h][nt][e] = 0.f;
+                }
+              }
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot]);
+        if (++slot == p.depth) {
+          slot = 0;
+          phase ^= 1;
+        }
+      }
+
+      // Reduce the SKW partial sums of each row tile in a fixed order.
+      const int per_tile = kBoxRows * M;
+#pragma unroll
+      for (int nt = 0; nt < MT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int m = 8 * nt + 2 * t + (e & 1);
+          const int r = g + 8 * (e >> 1);
+          if (m < M) red[(rt * p.SKW + sk) * per_tile + r * M + m] = y[nt][e];
+        }
+      named_barrier_sync(1, nthr);
+      for (int o = tid; o < p.RT * per_tile; o += nthr) {
+        const int rto = o / per_tile, rem = o % per_tile;
+        float sum = 0.f;
+        for (int s2 = 0; s2 < p.SKW; ++s2) sum += red[(rto * p.SKW + s2) * per_tile + rem];
+        if (csize == 1) {
+          const int row = (item * p.RT + rto) * kBoxRows + rem / M;
+          const int m = rem % M;
+          if (row < p.N) {
+            if (p.y_bf16)
+              reinterpret_cast<__nv_bfloat16*>(p.Y)[size_t(m) * p.N + row] = __float2bfloat16_rn(sum);
+            else
+              reinterpret_cast<float*>(p.Y)[size_t(m) * p.N + row] = sum;
+          }
+        } else {
+          part[size_t(local_item) * p.RT * per_tile + o] = sum;
+        }
+      }
+      named_barrier_sync(1, nthr);
+    }
+  }
+
+  if (csize > 1) {
+    // Add the ranks' partial sums in rank order through distributed shared
+    // memory; rank r writes the outputs with index % csize == r.
+    cluster_sync();
+    if (warp < kNumConsumerWarps) {
+      const int per_item = p.RT * kBoxRows * p.M;
+      int n_local = 0;
+      for (int item = cid; item < p.items; item += ncl) ++n_local;
+      const uint32_t part_local = smem_addr(smem + p.off_part);
+      for (int e = int(threadIdx.x) * int(csize) + int(rank); e < n_local * per_item;
+           e += kNumConsumerWarps * 32 * int(csize)) {
+        float sum = 0.f;
+        for (uint32_t r2 = 0; r2 < csize; ++r2)
+          sum += ld_dsmem_f32(map_to_rank(part_local + uint32_t(e) * 4, r2));
+        const int li = e / per_item, rem = e % per_item;
+        const int item = cid + li * ncl;
+        const int rto = rem / (kBoxRows * p.M), rr = rem % (kBoxRows * p.M);
+        const int row = (item * p.RT + rto) * kBoxRows + rr / p.M;
+        const int m = rr % p.M;
+        if (row < p.N) {
+          if (p.y_bf16)
+            reinterpret_cast<__nv_bfloat16*>(p.Y)[size_t(m) * p.N + row] = __float2bfloat16_rn(sum);
+          else
+            reinterpret_cast<float*>(p.Y)[size_t(m) * p.N + row] = sum;
+        }
+      }
+    }
+    cluster_sync();
+  }
+}
+
+}  // namespace gemv
+}  // namespace wq

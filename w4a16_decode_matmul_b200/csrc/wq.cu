@@ -1,0 +1,456 @@
+// wq.cu -- the C ABI declared in include/wq.h: argument checks, TMA
+// descriptor encoding, launch configuration, kernel dispatch.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "wq.h"
+#include "common.cuh"
+#include "quantize.cuh"
+#include "gemv.cuh"
+
+namespace {
+
+using wq::gemv::Params;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  int sms = 0;
+  int max_smem_optin = 0;
+};
+
+DeviceInfo g_devices[kMaxDevices];
+std::mutex g_mutex;
+
+bool device_info(DeviceInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceInfo& d = g_devices[dev];
+  if (d.sms == 0) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return false;
+    if (cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
+                               dev) != cudaSuccess)
+      return false;
+  }
+  *out = d;
+  return true;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [rows][cols] of `elem_bytes`-byte elements.
+bool encode_2d(CUtensorMap* map, const void* base, CUtensorMapDataType type, int elem_bytes,
+               uint64_t cols, uint64_t rows, uint32_t box_cols, uint32_t box_rows) {
+  auto fn = tensor_map_encoder();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * uint64_t(elem_bytes)};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, type, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_format(int64_t N, int64_t K, int bits, int group) {
+  if (bits != 4 && bits != 8) return false;
+  if (group != 32 && group != 64 && group != 128) return false;
+  if (N < 1 || K < 32 || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31)) return false;
+  if (K % 32 != 0 || K % group != 0) return false;
+  return true;
+}
+
+unsigned grid_for_elements(int64_t total, int sms) {
+  const int64_t warps_needed = (total + 1023) / 1024;
+  const int64_t blocks = (warps_needed + 7) / 8;
+  return unsigned(std::max<int64_t>(1, std::min<int64_t>(blocks, int64_t(sms) * 16)));
+}
+
+// ---------------------------------------------------------------- quantize
+
+template <int BITS, bool SYM, int G>
+cudaError_t launch_quantize(const void* W, int64_t total, void* codes, void* scales, void* zeros,
+                            cudaStream_t s, int sms) {
+  wq::quantize_kernel<BITS, SYM, G><<<grid_for_elements(total, sms), 256, 0, s>>>(
+      static_cast<const __half*>(W), total, static_cast<uint8_t*>(codes),
+      static_cast<__half*>(scales), static_cast<__half*>(zeros));
+  return cudaGetLastError();
+}
+
+template <int BITS, bool SYM, int G>
+cudaError_t launch_dequantize(const void* codes, const void* scales, const void* zeros,
+                              int64_t total, void* out, cudaStream_t s, int sms) {
+  wq::dequantize_kernel<BITS, SYM, G><<<grid_for_elements(total, sms), 256, 0, s>>>(
+      static_cast<const uint8_t*>(codes), static_cast<const __half*>(scales),
+      static_cast<const __half*>(zeros), total, static_cast<__nv_bfloat16*>(out));
+  return cudaGetLastError();
+}
+
+template <template <int, bool, int> class F, typename... Args>
+cudaError_t dispatch_format(int bits, bool sym, int group, Args... args) {
+#define WQ_CASE(B, S, G)                                        \
+  if (bits == B && sym == S && group == G) return F<B, S, G>::run(args...);
+  WQ_CASE(4, false, 32) WQ_CASE(4, false, 64) WQ_CASE(4, false, 128)
+  WQ_CASE(4, true, 32) WQ_CASE(4, true, 64) WQ_CASE(4, true, 128)
+  WQ_CASE(8, false, 32) WQ_CASE(8, false, 64) WQ_CASE(8, false, 128)
+  WQ_CASE(8, true, 32) WQ_CASE(8, true, 64) WQ_CASE(8, true, 128)
+#undef WQ_CASE
+  return cudaErrorInvalidValue;
+}
+
+template <int B, bool S, int G>
+struct QuantizeOp {
+  static cudaError_t run(const void* W, int64_t total, void* c, void* sc, void* z,
+                         cudaStream_t s, int sms) {
+    return launch_quantize<B, S, G>(W, total, c, sc, z, s, sms);
+  }
+};
+
+template <int B, bool S, int G>
+struct DequantizeOp {
+  static cudaError_t run(const void* c, const void* sc, const void* z, int64_t total, void* out,
+                         cudaStream_t s, int sms) {
+    return launch_dequantize<B, S, G>(c, sc, z, total, out, s, sms);
+  }
+};
+
+// ---------------------------------------------------------------- matmul
+
+struct GemvPlan {
+  Params p;
+  int C = 1;
+  int grid = 1;
+  size_t smem = 0;
+};
+
+template <int BITS, bool SYM, int G, int MT>
+const void* gemv_kernel_ptr() {
+  return reinterpret_cast<const void*>(&wq::gemv::gemv_kernel<BITS, SYM, G, MT>);
+}
+
+// Shared-memory layout and work split for one call with K split over C
+// cluster ranks and `bpw` boxes per warp and stage.  False if it does not fit
+// with at least `min_depth` ring stages.
+bool plan_gemv_with(int M, int N, int K, int bits, int group, const DeviceInfo& dev,
+                    int cluster_cap, int C, int bpw, int min_depth, GemvPlan* plan) {
+  auto round_up = [](int a, int b) { return (a + b - 1) / b * b; };
+  const int box_k = wq::gemv::kBoxRowBytes * 8 / bits;
+  const int granule = std::max(box_k, group);
+  const int tiles = (N + 15) / 16;
+  const size_t budget = size_t(dev.max_smem_optin);
+  const int MT = M <= 8 ? 1 : (M <= 16 ? 2 : 4);
+
+  const int kc = round_up((K + C - 1) / C, granule);
+  C = (K + kc - 1) / kc;  // ranks that have work
+  int skw = wq::gemv::kNumConsumerWarps;
+  while (skw > 1 && skw * box_k * bpw > kc) skw /= 2;
+  if (skw * box_k * bpw > kc && bpw > 1) return false;
+  const int RT = wq::gemv::kNumConsumerWarps / skw;
+  const int stage_k = skw * bpw * box_k;
+  const int sg = stage_k / group;
+  const int ngroups = K / group;
+
+  Params& p = plan->p;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.ngroups = ngroups;
+  p.row_tiles = tiles;
+  p.RT = RT;
+  p.SKW = skw;
+  p.BPW = bpw;
+  p.items = (tiles + RT - 1) / RT;
+  p.kc = kc;
+  p.stage_k = stage_k;
+  p.stages_per_item = (kc + stage_k - 1) / stage_k;
+  p.meta_tma = (ngroups % 8 == 0 && sg % 8 == 0 && (kc / group) % 8 == 0) ? 1 : 0;
+
+  const uint32_t codes_bytes = uint32_t(RT * skw * bpw * wq::gemv::kBoxBytes);
+  const uint32_t meta_bytes = uint32_t(2 * RT * 16 * sg * 2);  // scales + zeros
+  p.meta_offset = codes_bytes;
+  p.stage_bytes = uint32_t(round_up(int(codes_bytes + meta_bytes), 1024));
+
+  int clusters = std::max(1, dev.sms / C);
+  if (cluster_cap > 0) clusters = std::min(clusters, cluster_cap);
+  const int items_per_cluster_max = (p.items + clusters - 1) / clusters;
+  const size_t off = 1024;  // barriers + flags
+  const size_t fixed_x = size_t(round_up(kc * M * 2, 128));
+  const size_t fixed_sx = size_t(round_up((kc / group) * 8 * MT * 4, 128));
+  const size_t fixed_red = size_t(round_up(16 * 16 * M * 4, 128));
+  const size_t fixed_part =
+      C > 1 ? size_t(round_up(items_per_cluster_max * RT * 16 * M * 4, 128)) : 0;
+  const size_t fixed = off + fixed_x + fixed_sx + fixed_red + fixed_part;
+  if (fixed + size_t(min_depth) * p.stage_bytes > budget) return false;
+  int depth = int((budget - fixed) / p.stage_bytes);
+  depth = std::min(depth, 32);
+  // no point holding more stages than the CTA will ever consume
+  depth = std::min(depth, std::max(2, items_per_cluster_max * p.stages_per_item));
+  p.depth = depth;
+  p.off_ring = uint32_t(off);
+  p.off_x = uint32_t(off + size_t(depth) * p.stage_bytes);
+  p.off_sx = uint32_t(p.off_x + fixed_x);
+  p.off_red = uint32_t(p.off_sx + fixed_sx);
+  p.off_part = uint32_t(p.off_red + fixed_red);
+  plan->smem = p.off_part + fixed_part;
+  plan->C = C;
+  plan->grid = std::min(p.items, clusters) * C;
+  return true;
+}
+
+// Choose the cluster split and stage size.  K is split across a cluster when
+// there are too few row tiles to fill the SMs, or when the activations would
+// not fit in shared memory; stages shrink before the ring gets shallow.
+bool plan_gemv(int M, int N, int K, int bits, int group, const DeviceInfo& dev, int cluster_cap,
+               GemvPlan* plan) {
+  const int tiles = (N + 15) / 16;
+  const int sms = dev.sms;
+  int C0 = 1;
+  if (tiles < 3 * sms) C0 = 2;
+  if (tiles < sms) C0 = 4;
+  if (tiles < sms / 4) C0 = 8;
+  const int bpw_min = (bits == 8 && group == 128) ? 2 : 1;
+  const int bpw_max = bits == 8 ? 4 : 2;
+  for (int min_depth : {3, 2}) {
+    for (int C = C0; C <= 16; C *= 2) {
+      const int box_k = wq::gemv::kBoxRowBytes * 8 / bits;
+      const int granule = std::max(box_k, group);
+      const int kc = (((K + C - 1) / C) + granule - 1) / granule * granule;
+      if (size_t(kc) * M * 2 > 128 * 1024 && C < 16) continue;
+      for (int bpw = bpw_max; bpw >= bpw_min; bpw /= 2)
+        if (plan_gemv_with(M, N, K, bits, group, dev, cluster_cap, C, bpw, min_depth, plan))
+          return true;
+    }
+  }
+  return false;
+}
+
+template <int BITS, bool SYM, int G, int MT>
+cudaError_t launch_gemv_t(GemvPlan& plan, const DeviceInfo& dev, const void* codes,
+                          const void* scales, const void* zeros, cudaStream_t s) {
+  auto kernel = &wq::gemv::gemv_kernel<BITS, SYM, G, MT>;
+  static int configured_smem[kMaxDevices] = {};  // per instantiation and device
+  int device = 0;
+  cudaGetDevice(&device);
+  if (device < 0 || device >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (configured_smem[device] == 0) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         dev.max_smem_optin);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+    configured_smem[device] = dev.max_smem_optin;
+  }
+
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attrs[1];
+  cfg.blockDim = dim3(wq::gemv::kThreads, 1, 1);
+  cfg.stream = s;
+  if (plan.C > 1) {
+    // Size the grid to the clusters that can be resident at once.
+    attrs[0].id = cudaLaunchAttributeClusterDimension;
+    attrs[0].val.clusterDim.x = unsigned(plan.C);
+    attrs[0].val.clusterDim.y = 1;
+    attrs[0].val.clusterDim.z = 1;
+    cfg.attrs = attrs;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(unsigned(plan.grid), 1, 1);
+    cfg.dynamicSmemBytes = plan.smem;
+    int max_clusters = 0;
+    cudaError_t e = cudaOccupancyMaxActiveClusters(&max_clusters, kernel, &cfg);
+    if (e != cudaSuccess) return e;
+    if (max_clusters < 1) return cudaErrorNotSupported;
+    if (plan.grid / plan.C > max_clusters) {
+      const Params keep = plan.p;
+      if (!plan_gemv(keep.M, keep.N, keep.K, BITS, G, dev, max_clusters, &plan))
+        return cudaErrorNotSupported;
+      plan.p.X = keep.X;
+      plan.p.Y = keep.Y;
+      plan.p.scales = keep.scales;
+      plan.p.zeros = keep.zeros;
+      plan.p.y_bf16 = keep.y_bf16;
+    }
+  }
+  cfg.gridDim = dim3(unsigned(plan.grid), 1, 1);
+  cfg.dynamicSmemBytes = plan.smem;
+
+  const Params& p = plan.p;
+  const int row_bytes = p.K * BITS / 8;
+  CUtensorMap tc, ts, tz;
+  const int sg = p.stage_k / G;
+  if (!encode_2d(&tc, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(row_bytes),
+                 uint64_t(p.N), wq::gemv::kBoxRowBytes, wq::gemv::kBoxRows))
+    return cudaErrorInvalidValue;
+  std::memcpy(&ts, &tc, sizeof(tc));
+  std::memcpy(&tz, &tc, sizeof(tc));
+  if (p.meta_tma) {
+    if (!encode_2d(&ts, scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, uint64_t(p.ngroups),
+                   uint64_t(p.N), uint32_t(sg), wq::gemv::kBoxRows))
+      return cudaErrorInvalidValue;
+    if (!SYM && !encode_2d(&tz, zeros, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, uint64_t(p.ngroups),
+                           uint64_t(p.N), uint32_t(sg), wq::gemv::kBoxRows))
+      return cudaErrorInvalidValue;
+  }
+  return cudaLaunchKernelEx(&cfg, kernel, tc, ts, tz, p);
+}
+
+template <int BITS, bool SYM, int G>
+struct GemvOp {
+  static cudaError_t run(GemvPlan* plan, const DeviceInfo* dev, const void* c, const void* sc,
+                         const void* z, cudaStream_t s) {
+    const int M = plan->p.M;
+    if (M <= 8) return launch_gemv_t<BITS, SYM, G, 1>(*plan, *dev, c, sc, z, s);
+    if (M <= 16) return launch_gemv_t<BITS, SYM, G, 2>(*plan, *dev, c, sc, z, s);
+    return launch_gemv_t<BITS, SYM, G, 4>(*plan, *dev, c, sc, z, s);
+  }
+};
+
+wq_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return WQ_OK;
+  if (e == cudaErrorInvalidValue) return WQ_ERR_INVALID_ARG;
+  if (e == cudaErrorNotSupported) return WQ_ERR_UNSUPPORTED;
+  return WQ_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t wq_codes_bytes(int64_t N, int64_t K, int bits) {
+  if ((bits != 4 && bits != 8) || N < 1 || K < 1 || (K * bits) % 8 != 0) return 0;
+  return size_t(N) * size_t(K) * size_t(bits) / 8;
+}
+
+size_t wq_meta_elems(int64_t N, int64_t K, int group) {
+  if (group < 1 || N < 1 || K < 1 || K % group != 0) return 0;
+  return size_t(N) * size_t(K / group);
+}
+
+wq_status wq_quantize(const void* W, int64_t N, int64_t K, int bits, int group, int symmetric,
+                      void* codes, void* scales, void* zeros, wq_stream_t stream) {
+  if (!valid_format(N, K, bits, group)) return WQ_ERR_INVALID_ARG;
+  if (symmetric != 0 && symmetric != 1) return WQ_ERR_INVALID_ARG;
+  if (!W || !codes || !scales || (symmetric ? zeros != nullptr : zeros == nullptr))
+    return WQ_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(codes) || !aligned16(scales) || (zeros && !aligned16(zeros)))
+    return WQ_ERR_ALIGNMENT;
+  DeviceInfo dev;
+  if (!device_info(&dev)) return WQ_ERR_CUDA;
+  const cudaError_t e = dispatch_format<QuantizeOp>(bits, symmetric != 0, group, W, N * K, codes,
+                                                    scales, zeros,
+                                                    reinterpret_cast<cudaStream_t>(stream), dev.sms);
+  return from_cuda(e);
+}
+
+wq_status wq_dequantize(const void* codes, const void* scales, const void* zeros, int64_t N,
+                        int64_t K, int bits, int group, int symmetric, void* W_out,
+                        wq_stream_t stream) {
+  if (!valid_format(N, K, bits, group)) return WQ_ERR_INVALID_ARG;
+  if (symmetric != 0 && symmetric != 1) return WQ_ERR_INVALID_ARG;
+  if (!W_out || !codes || !scales || (symmetric ? zeros != nullptr : zeros == nullptr))
+    return WQ_ERR_INVALID_ARG;
+  if (!aligned16(W_out) || !aligned16(codes) || !aligned16(scales) ||
+      (zeros && !aligned16(zeros)))
+    return WQ_ERR_ALIGNMENT;
+  DeviceInfo dev;
+  if (!device_info(&dev)) return WQ_ERR_CUDA;
+  const cudaError_t e =
+      dispatch_format<DequantizeOp>(bits, symmetric != 0, group, codes, scales, zeros, N * K,
+                                    W_out, reinterpret_cast<cudaStream_t>(stream), dev.sms);
+  return from_cuda(e);
+}
+
+wq_status wq_matmul(const void* X, int64_t M, const void* codes, const void* scales,
+                    const void* zeros, int64_t N, int64_t K, int bits, int group, int symmetric,
+                    void* Y, int out_dtype, wq_stream_t stream) {
+  if (!valid_format(N, K, bits, group) || M < 1 || M >= (int64_t(1) << 31))
+    return WQ_ERR_INVALID_ARG;
+  if (symmetric != 0 && symmetric != 1) return WQ_ERR_INVALID_ARG;
+  if (out_dtype != WQ_OUT_F32 && out_dtype != WQ_OUT_BF16) return WQ_ERR_INVALID_ARG;
+  if (!X || !codes || !scales || !Y || (symmetric ? zeros != nullptr : zeros == nullptr))
+    return WQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(codes) || !aligned16(scales) || !aligned16(Y) ||
+      (zeros && !aligned16(zeros)))
+    return WQ_ERR_ALIGNMENT;
+  if (M > 32) return WQ_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  if (!device_info(&dev)) return WQ_ERR_CUDA;
+  GemvPlan plan;
+  if (!plan_gemv(int(M), int(N), int(K), bits, group, dev, 0, &plan)) return WQ_ERR_UNSUPPORTED;
+  plan.p.X = static_cast<const __nv_bfloat16*>(X);
+  plan.p.Y = Y;
+  plan.p.scales = static_cast<const __half*>(scales);
+  plan.p.zeros = static_cast<const __half*>(zeros);
+  plan.p.y_bf16 = out_dtype == WQ_OUT_BF16;
+  const cudaError_t e = dispatch_format<GemvOp>(bits, symmetric != 0, group, &plan, &dev, codes,
+                                                scales, zeros,
+                                                reinterpret_cast<cudaStream_t>(stream));
+  return from_cuda(e);
+}
+
+wq_status wq_get_device_error(wq_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return WQ_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, wq::g_status, sizeof(v)) != cudaSuccess) return WQ_ERR_CUDA;
+  const unsigned int zero = 0;
+  if (cudaMemcpyToSymbol(wq::g_status, &zero, sizeof(zero)) != cudaSuccess) return WQ_ERR_CUDA;
+  return static_cast<wq_status>(v);
+}
+
+const char* wq_status_string(wq_status status) {
+  switch (status) {
+    case WQ_OK: return "ok";
+    case WQ_ERR_INVALID_ARG: return "invalid argument";
+    case WQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case WQ_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case WQ_ERR_CUDA: return "CUDA runtime error";
+    case WQ_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* wq_version(void) { return "wq 0.1.0 (sm_100a)"; }
+
+// Test hook, not part of the public ABI: the matmul plan for a device with
+// `sms` SMs and `smem_optin` bytes of shared memory per block, written to
+// out[0..23] (see tests/test_plan.py for the field order).  Returns 0 if no
+// plan exists.
+int wq_internal_plan_gemv(int M, int N, int K, int bits, int group, int sms, int smem_optin,
+                          int cluster_cap, int64_t* out) {
+  DeviceInfo dev;
+  dev.sms = sms;
+  dev.max_smem_optin = smem_optin;
+  GemvPlan plan;
+  if (!plan_gemv(M, N, K, bits, group, dev, cluster_cap, &plan)) return 0;
+  const Params& p = plan.p;
+  const int64_t v[] = {p.M,       p.N,           p.K,         p.ngroups,     p.row_tiles,
+                       p.items,   p.RT,          p.SKW,       p.BPW,         p.depth,
+                       p.kc,      p.stage_k,     p.stages_per_item, p.meta_tma, p.stage_bytes,
+                       p.meta_offset, p.off_ring, p.off_x,    p.off_sx,      p.off_red,
+                       p.off_part, int64_t(plan.smem), plan.C, plan.grid};
+  for (size_t i = 0; i < sizeof(v) / sizeof(v[0]); ++i) out[i] = v[i];
+  return 1;
+}
+
+}  // extern "C"
