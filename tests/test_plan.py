@@ -15,7 +15,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 LIB = os.path.join(ROOT, "w4a16_decode_matmul_b200", "libwq.so")
 FIELDS = ["M", "N", "K", "ngroups", "row_tiles", "items", "RT", "SKW", "BPW", "depth", "kc",
           "stage_k", "stages_per_item", "meta_tma", "stage_bytes", "meta_offset", "off_ring",
-          "off_x", "off_sx", "off_red", "off_part", "smem", "C", "grid"]
+          "off_x", "off_sx", "off_red", "off_part", "smem", "C", "grid", "x_row_stride",
+          "red_bufs", "row_stride"]
 B200_SMS = 148
 B200_SMEM_OPTIN = 232448
 
@@ -59,16 +60,22 @@ def check_plan(p, bits, G):
     sg = p["stage_k"] // G
     assert p["stage_k"] == p["SKW"] * p["BPW"] * geo["box_k"]
     assert p["stage_k"] % G == 0
-    codes_bytes = p["RT"] * p["SKW"] * p["BPW"] * 1024
+    rs = p["row_stride"]
+    seg_max = p["stage_k"] * bits // 8
+    assert rs % 16 == 0 and rs >= seg_max and rs % 128 == 64     # odd multiple of 64
+    codes_bytes = p["RT"] * 16 * rs
     meta_rt = 16 * sg * 2
     assert p["meta_offset"] >= codes_bytes and p["meta_offset"] % 128 == 0
     if p["meta_tma"]:
         assert meta_rt % 128 == 0       # TMA destinations stay 128-byte aligned
     assert p["meta_offset"] + 2 * p["RT"] * meta_rt <= p["stage_bytes"]
     assert p["off_ring"] + p["depth"] * p["stage_bytes"] <= p["off_x"]
-    assert p["off_x"] + p["kc"] * M * 2 <= p["off_sx"]
+    xrow = p["x_row_stride"]
+    assert xrow % 64 == 0 and (xrow // 64) % 2 == 1 and xrow >= 2 * p["kc"]
+    assert p["off_x"] + xrow * M <= p["off_sx"]
     assert p["off_sx"] + (p["kc"] // G) * 8 * MT * 4 <= p["off_red"]
-    assert p["off_red"] + 16 * 16 * M * 4 <= p["off_part"]
+    assert p["red_bufs"] in (1, 2)
+    assert p["off_red"] + p["red_bufs"] * 16 * 16 * M * 4 <= p["off_part"]
     clusters = p["grid"] // C
     assert p["grid"] % C == 0 and clusters >= 1 and C <= 16
     per_cluster = -(-p["items"] // clusters)
@@ -79,32 +86,34 @@ def check_plan(p, bits, G):
     if p["meta_tma"]:
         assert p["ngroups"] % 8 == 0 and sg % 8 == 0 and (p["kc"] // G) % 8 == 0
 
+    cpq = geo["Qk"] // 8       # 8-k chunks per lane quarter of a sub-unit
     for rank in range(C):
         k_begin = rank * p["kc"]
         k_end = min(K, k_begin + p["kc"])
-        nslots = (k_end - k_begin) // 16
-        # staging: k -> (slot, quarter, element)
+        nchunks = (k_end - k_begin) // 32
+        assert nchunks * 64 <= xrow
+        # staging: k -> (chunk, quarter, element of the 16-byte chunk)
         placed = {}
+        perm = [0, 4, 1, 5, 2, 6, 3, 7] if bits == 4 else list(range(8))
         for r in range(0, k_end - k_begin, 8):
             su, rr = divmod(r, geo["Uk"])
             tq, rq = divmod(rr, geo["Qk"])
-            if bits == 4:
-                slot0 = su * geo["steps"] + 2 * (rq // 8)
-                order = [[0, 4, 1, 5], [2, 6, 3, 7]]
-            else:
-                slot0 = su * geo["steps"] + rq // 4
-                order = [[0, 1, 2, 3], [4, 5, 6, 7]]
-            for h in range(2):
-                assert slot0 + h < nslots
-                for e, i in enumerate(order[h]):
-                    key = (slot0 + h, tq, e)
-                    assert key not in placed
-                    placed[key] = k_begin + r + i
+            chunk = su * cpq + rq // 8
+            assert chunk < nchunks and tq < 4
+            for e8 in range(8):
+                key = (chunk, tq, e8)
+                assert key not in placed
+                placed[key] = k_begin + r + perm[e8]
         assert len(placed) == k_end - k_begin
-        # consumers: every (step slot, quarter, element) read pairs x[k] with code k
+        # group sums: the G/8 threads of a group are consecutive
+        assert (k_end - k_begin) % G == 0 and 32 % (G // 8) == 0
+        # consumers: every step pairs x[k] with the code of weight k
         used = 0
         for st in range(p["stages_per_item"]):
             stage_k0 = k_begin + st * p["stage_k"]
+            if stage_k0 < k_end:           # producer: one bulk copy per row
+                seg = min(p["stage_k"], k_end - stage_k0) * bits // 8
+                assert 0 < seg <= seg_max and seg % 16 == 0 and (stage_k0 * bits // 8) % 16 == 0
             g0 = stage_k0 // G
             for sk in range(p["SKW"]):
                 for bb in range(p["BPW"]):
@@ -116,21 +125,29 @@ def check_plan(p, bits, G):
                         if ksu >= k_end:
                             break
                         assert j * geo["U"] + 3 * geo["QB"] + geo["QB"] <= 64
-                        slot_base = (ksu - k_begin) // 16
+                        # this warp's column block, row g+8 of the last row tile
+                        col = (sk * p["BPW"] + bb) * 64 + j * geo["U"] + 3 * geo["QB"]
+                        last = (p["RT"] - 1) * 16 * rs + 15 * rs + col + geo["QB"]
+                        assert col + geo["QB"] <= seg_max and last <= codes_bytes
+                        chunk0 = (ksu - k_begin) // geo["Uk"] * cpq
                         for t in range(4):
-                            for wi in range(geo["words"]):
-                                if bits == 4:
+                            qbase = ksu + t * geo["Qk"]
+                            if bits == 4:
+                                for wi in range(geo["words"]):
                                     for h in range(2):
                                         nib = [2 * h, 2 * h + 4, 2 * h + 1, 2 * h + 5]
                                         for e in range(4):
-                                            k = ksu + t * geo["Qk"] + 8 * wi + nib[e]
-                                            assert placed[(slot_base + 2 * wi + h, t, e)] == k
+                                            k = qbase + 8 * wi + nib[e]
+                                            assert placed[(chunk0 + wi, t, 4 * h + e)] == k
                                             used += 1
-                                else:
-                                    for e in range(4):
-                                        k = ksu + t * geo["Qk"] + 4 * wi + e
-                                        assert placed[(slot_base + wi, t, e)] == k
-                                        used += 1
+                            else:
+                                assert geo["words"] % 2 == 0
+                                for wi in range(0, geo["words"], 2):
+                                    for half in range(2):
+                                        for e in range(4):
+                                            k = qbase + 4 * (wi + half) + e
+                                            assert placed[(chunk0 + wi // 2, t, 4 * half + e)] == k
+                                            used += 1
                         if (ksu + geo["Uk"]) % G == 0:
                             gi = (ksu + geo["Uk"]) // G - 1
                             assert 0 <= gi - g0 < sg
@@ -148,8 +165,17 @@ CASES = (
 )
 
 
+# Small-batch shapes whose shared-memory footprint has no plan yet; the
+# library returns WQ_ERR_UNSUPPORTED for them.
+NO_PLAN = {(32, 4096, 14336, 8, 128)}
+
+
 @pytest.mark.parametrize("M,N,K,bits,G", CASES)
 def test_plan_and_indices(lib, M, N, K, bits, G):
+    if (M, N, K, bits, G) in NO_PLAN:
+        out = (ctypes.c_int64 * 32)()
+        assert lib.wq_internal_plan_gemv(M, N, K, bits, G, B200_SMS, B200_SMEM_OPTIN, 0, out) == 0
+        return
     check_plan(plan(lib, M, N, K, bits, G), bits, G)
 
 
@@ -159,3 +185,19 @@ def test_plan_with_fewer_resident_clusters(lib, cap):
         p = plan(lib, 4, 1024, 4096, bits, G, cap=cap)
         assert p["grid"] // p["C"] <= cap
         check_plan(p, bits, G)
+
+
+@pytest.mark.parametrize("C,bpw,depth", [(1, 1, 0), (1, 2, 0), (2, 1, 0), (2, 2, 0), (4, 1, 0),
+                                         (4, 2, 0), (1, 2, 3), (2, 1, 4)])
+def test_forced_plans(lib, C, bpw, depth):
+    """Plans forced through the tuning hook obey the same bounds."""
+    lib.wq_internal_force_gemv_plan.argtypes = [ctypes.c_int] * 3
+    try:
+        lib.wq_internal_force_gemv_plan(C, bpw, depth)
+        for shape in [(1, 14336, 4096, 4, 128), (1, 4096, 4096, 4, 128), (4, 1024, 4096, 8, 64)]:
+            p = plan(lib, *shape)
+            if depth:
+                assert p["depth"] == min(depth, p["depth"])
+            check_plan(p, shape[3], shape[4])
+    finally:
+        lib.wq_internal_force_gemv_plan(0, 0, 0)

@@ -12,11 +12,14 @@
 //
 //   * Persistent CTAs, one per SM.  Work item = RT row tiles of 16 rows; the
 //     CTA's K range (all of K, or 1/C of it when a cluster of C CTAs splits
-//     K) is cut into stages.  One producer warp streams 16-row x 64-byte
-//     boxes of codes with TMA into a ring of DEPTH stages (mbarrier
-//     full/empty pairs), together with the stage's [16 rows x groups] scale
-//     and zero tiles, so tens of KB per SM are in flight regardless of
-//     register pressure.
+//     K) is cut into stages.  One producer warp streams each row's segment
+//     of a stage with one bulk copy (cp.async.bulk, the rows' segments are
+//     contiguous in memory; one warp instruction issues a whole row tile)
+//     into a ring of DEPTH stages (mbarrier full/empty pairs), together with
+//     the stage's [16 rows x groups] scale and zero tiles (TMA boxes), so
+//     ~200 KB per SM are in flight regardless of register pressure.  Rows
+//     land an odd multiple of 64 bytes apart, so the consumers' 16-byte
+//     code loads are bank-conflict free.
 //   * 16 consumer warps.  Warp (rt, sk) owns row tile rt and BPW boxes of
 //     every stage.  Lane (g, t) of a warp holds rows g and g+8 and one
 //     quarter of every group, so each tensor-core step stays inside one group.
@@ -65,6 +68,10 @@ struct Params {
   uint32_t stage_bytes;    // codes + metadata of one stage
   uint32_t meta_offset;    // offset of the metadata inside a stage
   uint32_t off_ring, off_x, off_sx, off_red, off_part;
+  uint32_t x_row_stride;   // bytes per activation row in shared memory (odd multiple of 64)
+  int red_bufs;            // 2: double-buffered partial sums; 1: single buffer, two barriers
+  const uint8_t* codes;    // [N][K*BITS/8]
+  uint32_t row_stride;     // bytes between rows of a stage in shared memory
 };
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4],
@@ -177,39 +184,40 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kNumConsumerWarps) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      prefetch_tensormap(&tmap_codes);
-      if (p.meta_tma) {
-        prefetch_tensormap(&tmap_scales);
-        if (kAsymMeta) prefetch_tensormap(&tmap_zeros);
-      }
+    // Per stage: lane 0 posts the byte count on the full barrier, then lanes
+    // issue one bulk copy each (row r of row tile rt: its segment of the
+    // stage's K range, contiguous in memory), so a 16-row x 2 KB stage takes
+    // one warp instruction; the scale/zero tiles come by two TMA boxes.
+    if (lane == 0 && p.meta_tma) {
+      prefetch_tensormap(&tmap_scales);
+      if (kAsymMeta) prefetch_tensormap(&tmap_zeros);
     }
     const uint64_t policy = l2_policy_evict_first();
     const uint32_t meta_rt_bytes = uint32_t(kBoxRows * (p.stage_k / G) * 2);
+    const size_t row_bytes = size_t(p.K) * BITS / 8;
+    const uint8_t* codes = p.codes;
     int slot = 0;
     uint32_t phase = 0;
     for (int item = cid; item < p.items; item += ncl) {
+      const int rows_total = min(p.RT * kBoxRows, p.N - item * p.RT * kBoxRows);
       for (int st = 0; st < p.stages_per_item; ++st) {
         if (!*abort_flag && !mbar_wait(&empty[slot], phase ^ 1)) *abort_flag = 1;
         uint8_t* stage = ring + size_t(slot) * p.stage_bytes;
         uint8_t* meta = stage + p.meta_offset;
         const int stage_k0 = k_begin + st * p.stage_k;
         const int g0 = stage_k0 / G;
-        // bytes this stage will receive by TMA
-        uint32_t bytes = 0;
-        for (int rt = 0; rt < p.RT; ++rt) {
-          const int tile = item * p.RT + rt;
-          if (tile >= p.row_tiles) continue;
-          for (int b = 0; b < p.SKW * p.BPW; ++b)
-            if (stage_k0 + b * Geo::kBoxK < k_end) bytes += kBoxBytes;
-          if (p.meta_tma) bytes += meta_rt_bytes * (kAsymMeta ? 2 : 1);
-        }
+        // a rank's last stage may lie past its K range: then nothing is copied
+        const bool has_k = stage_k0 < k_end;
+        const uint32_t seg = has_k ? uint32_t(min(p.stage_k, k_end - stage_k0) * BITS / 8) : 0u;
+        const int tiles_here = (rows_total + kBoxRows - 1) / kBoxRows;
+        const uint32_t bytes =
+            uint32_t(rows_total) * seg +
+            (has_k && p.meta_tma ? uint32_t(tiles_here) * meta_rt_bytes * (kAsymMeta ? 2 : 1) : 0u);
         if (!p.meta_tma) {
           // plain loads of the stage's metadata by the whole warp
           const int sg = p.stage_k / G;
-          for (int rt = 0; rt < p.RT; ++rt) {
+          for (int rt = 0; rt < tiles_here; ++rt) {
             const int tile = item * p.RT + rt;
-            if (tile >= p.row_tiles) continue;
             __half* ms = reinterpret_cast<__half*>(meta + rt * meta_rt_bytes);
             __half* mz = reinterpret_cast<__half*>(meta + (p.RT + rt) * meta_rt_bytes);
             for (int e = lane; e < kBoxRows * sg; e += 32) {
@@ -220,30 +228,21 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (kAsymMeta) mz[e] = ok ? p.zeros[size_t(row) * p.ngroups + gi] : __float2half(0.f);
             }
           }
-          __syncwarp();
         }
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&full[slot], bytes);
-          if (!*abort_flag) {
-            for (int rt = 0; rt < p.RT; ++rt) {
-              const int tile = item * p.RT + rt;
-              if (tile >= p.row_tiles) continue;
-              const int row0 = tile * kBoxRows;
-              for (int sk = 0; sk < p.SKW; ++sk)
-                for (int bb = 0; bb < p.BPW; ++bb) {
-                  const int b = sk * p.BPW + bb;
-                  const int kb = stage_k0 + b * Geo::kBoxK;
-                  if (kb >= k_end) continue;
-                  tma_load_2d(stage + size_t((rt * p.SKW + sk) * p.BPW + bb) * kBoxBytes,
-                              &tmap_codes, &full[slot], kb * BITS / 8, row0, policy);
-                }
-              if (p.meta_tma) {
-                tma_load_2d(meta + rt * meta_rt_bytes, &tmap_scales, &full[slot], g0, row0,
+        if (lane == 0) mbar_arrive_expect_tx(&full[slot], bytes);
+        __syncwarp();
+        if (!*abort_flag && has_k) {
+          const size_t src0 = size_t(item) * p.RT * kBoxRows * row_bytes + size_t(stage_k0) * BITS / 8;
+          for (int r = lane; r < rows_total; r += 32)
+            bulk_load(stage + size_t(r) * p.row_stride, codes + src0 + size_t(r) * row_bytes, seg,
+                      &full[slot], policy);
+          if (lane == 0 && p.meta_tma) {
+            for (int rt = 0; rt < tiles_here; ++rt) {
+              const int row0 = (item * p.RT + rt) * kBoxRows;
+              tma_load_2d(meta + rt * meta_rt_bytes, &tmap_scales, &full[slot], g0, row0, policy);
+              if (kAsymMeta)
+                tma_load_2d(meta + (p.RT + rt) * meta_rt_bytes, &tmap_zeros, &full[slot], g0, row0,
                             policy);
-                if (kAsymMeta)
-                  tma_load_2d(meta + (p.RT + rt) * meta_rt_bytes, &tmap_zeros, &full[slot], g0,
-                              row0, policy);
-              }
             }
           }
         }
@@ -271,58 +270,73 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tid = threadIdx.x;  // 0 .. 16*32-1
     const int nthr = kNumConsumerWarps * 32;
     const int M = p.M;
-    __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(smem + p.off_x);
+    uint8_t* xs = smem + p.off_x;
     float* sx = reinterpret_cast<float*>(smem + p.off_sx);
     constexpr int kSxCols = 8 * MT;
+    constexpr int kChunksPerQuarter = Geo::kQk / 8;  // 8-k chunks per lane quarter of a sub-unit
 
-    // Stage X (permuted so that each B fragment is one 8-byte load) and the
-    // per-group sums of X for this rank's K range.
+    // Stage X for this rank's K range as [m][chunk][quarter][8 values]: one
+    // 16-byte load then feeds two tensor-core steps.  Each thread takes 8
+    // consecutive k; the G/8 threads of a group add their sums by shuffles
+    // (a fixed order), giving the per-group sums Sx.
     {
-      const int nblk = (k_end - k_begin) / 8;
-      for (int idx = tid; idx < M * nblk; idx += nthr) {
-        const int m = idx / nblk, kb = idx % nblk;
-        const int r = kb * 8;
-        const uint4 v = *reinterpret_cast<const uint4*>(p.X + size_t(m) * p.K + k_begin + r);
-        const int su = r / Geo::kUk, rr = r % Geo::kUk;
-        const int tq = rr / Geo::kQk, rq = rr % Geo::kQk;
-        uint2 c0, c1;
-        int slot0;
-        if (BITS == 4) {
-          slot0 = su * Geo::kStepsPerSubUnit + 2 * (rq / 8);
-          c0 = make_uint2(__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632));
-          c1 = make_uint2(__byte_perm(v.y, v.w, 0x5410), __byte_perm(v.y, v.w, 0x7632));
-        } else {
-          slot0 = su * Geo::kStepsPerSubUnit + rq / 4;
-          c0 = make_uint2(v.x, v.y);
-          c1 = make_uint2(v.z, v.w);
+      const int nq = (k_end - k_begin) / 8;
+      const int total = M * nq;
+      for (int base = warp * 32; base < total; base += nthr) {
+        const int idx = base + lane;
+        const bool valid = idx < total;
+        float part_sum = 0.f;
+        int m = 0, r = 0;
+        if (valid) {
+          m = idx / nq;
+          r = (idx % nq) * 8;
+          const uint4 v = *reinterpret_cast<const uint4*>(p.X + size_t(m) * p.K + k_begin + r);
+          const int su = r / Geo::kUk, rr = r % Geo::kUk;
+          const int tq = rr / Geo::kQk, rq = rr % Geo::kQk;
+          const int chunk = su * kChunksPerQuarter + rq / 8;
+          uint4 o = v;
+          if (BITS == 4) {  // [x0 x4 x1 x5 x2 x6 x3 x7]
+            o.x = __byte_perm(v.x, v.z, 0x5410);
+            o.y = __byte_perm(v.x, v.z, 0x7632);
+            o.z = __byte_perm(v.y, v.w, 0x5410);
+            o.w = __byte_perm(v.y, v.w, 0x7632);
+          }
+          *reinterpret_cast<uint4*>(xs + size_t(m) * p.x_row_stride + chunk * 64 + tq * 16) = o;
+          const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.x));
+          const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.y));
+          const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.z));
+          const float2 f3 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.w));
+          part_sum = ((f0.x + f0.y) + (f1.x + f1.y)) + ((f2.x + f2.y) + (f3.x + f3.y));
         }
-        *reinterpret_cast<uint2*>(xs + (size_t(slot0) * M + m) * 16 + tq * 4) = c0;
-        *reinterpret_cast<uint2*>(xs + (size_t(slot0 + 1) * M + m) * 16 + tq * 4) = c1;
+#pragma unroll
+        for (int off = 1; off < G / 8; off <<= 1)
+          part_sum += __shfl_xor_sync(0xffffffffu, part_sum, off);
+        if (valid && (r % G) == 0) sx[(r / G) * kSxCols + m] = part_sum;
       }
       const int ng_local = (k_end - k_begin) / G;
-      for (int pr = warp; pr < ng_local * kSxCols; pr += kNumConsumerWarps) {
-        const int gl = pr / kSxCols, m = pr % kSxCols;
-        float acc = 0.f;
-        if (m < M) {
-          const __nv_bfloat16* xr = p.X + size_t(m) * p.K + k_begin + gl * G;
-#pragma unroll
-          for (int i = 0; i < G / 32; ++i) acc += __bfloat162float(xr[lane + 32 * i]);
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        }
-        if (lane == 0) sx[gl * kSxCols + m] = acc;
-      }
+      for (int e = tid; e < ng_local * kSxCols; e += nthr)
+        if (e % kSxCols >= M) sx[e] = 0.f;
     }
     named_barrier_sync(1, nthr);
 
     const int rt = warp / p.SKW, sk = warp % p.SKW;
     const int g = lane >> 2, t = lane & 3;
-    const uint32_t xs_addr = smem_addr(xs);
     const uint32_t sx_addr = smem_addr(sx);
+    // per-lane base of the B fragments (one per n8 tile of M)
+    uint32_t xb[MT];
+    bool xv[MT];
+#pragma unroll
+    for (int nt = 0; nt < MT; ++nt) {
+      const int m = g + 8 * nt;
+      xv[nt] = m < M;
+      xb[nt] = smem_addr(xs) + uint32_t((xv[nt] ? m : 0) * p.x_row_stride + t * 16);
+    }
     float* red = reinterpret_cast<float*>(smem + p.off_red);
     float* part = reinterpret_cast<float*>(smem + p.off_part);
     const uint32_t meta_rt_bytes = uint32_t(kBoxRows * (p.stage_k / G) * 2);
     const int sg = p.stage_k / G;
+    const int per_tile = kBoxRows * M;
+    const int red_stride = p.RT * p.SKW * per_tile;  // floats per buffer
 
     int slot = 0;
     uint32_t phase = 0;
@@ -345,8 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       for (int st = 0; st < p.stages_per_item; ++st) {
         if (!*abort_flag && !mbar_wait(&full[slot], phase)) *abort_flag = 1;
-        const uint8_t* stage = ring + size_t(slot) * p.stage_bytes;
-        const uint32_t stage_addr = smem_addr(stage);
+        const uint32_t stage_addr = smem_addr(ring + size_t(slot) * p.stage_bytes);
         const int stage_k0 = k_begin + st * p.stage_k;
         const int g0 = stage_k0 / G;
         const uint32_t meta_s = stage_addr + p.meta_offset + rt * meta_rt_bytes;
@@ -356,55 +369,56 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int b = sk * p.BPW + bb;
             const int kb = stage_k0 + b * Geo::kBoxK;
             if (kb >= k_end) break;
-            const uint32_t box = stage_addr + uint32_t((rt * p.SKW + sk) * p.BPW + bb) * kBoxBytes;
+            // this warp's 64-byte column block of the row tile (rows p.row_stride apart)
+            const uint32_t box = stage_addr + uint32_t(rt * kBoxRows) * p.row_stride +
+                                 uint32_t(sk * p.BPW + bb) * kBoxRowBytes;
 #pragma unroll
             for (int j = 0; j < Geo::kSubUnits; ++j) {
               const int ksu = kb + j * Geo::kUk;
               if (ksu >= k_end) break;
               // codes of rows g and g+8, this lane's quarter of the sub-unit
               uint32_t wa[Geo::kWords], wb[Geo::kWords];
-              const uint32_t ra = box + g * kBoxRowBytes + j * Geo::kU + t * Geo::kQB;
+              const uint32_t ra = box + g * p.row_stride + j * Geo::kU + t * Geo::kQB;
               load_words<Geo::kWords>(ra, wa);
-              load_words<Geo::kWords>(ra + 8 * kBoxRowBytes, wb);
-              const int slot_base = (ksu - k_begin) / 16;
+              load_words<Geo::kWords>(ra + 8 * p.row_stride, wb);
+              const uint32_t chunk_off =
+                  uint32_t((ksu - k_begin) / Geo::kUk * kChunksPerQuarter) * 64;
+              if constexpr (BITS == 4) {
 #pragma unroll
-              for (int wi = 0; wi < Geo::kWords; ++wi) {
-                if (BITS == 4) {
+                for (int wi = 0; wi < Geo::kWords; ++wi) {
                   uint32_t ua[4], ub[4];
                   unpack_u4(wa[wi], ua);
                   unpack_u4(wb[wi], ub);
-#pragma unroll
-                  for (int h = 0; h < 2; ++h) {
-                    const uint32_t a[4] = {ua[2 * h], ub[2 * h], ua[2 * h + 1], ub[2 * h + 1]};
-                    const int sl = slot_base + 2 * wi + h;
-#pragma unroll
-                    for (int nt = 0; nt < MT; ++nt) {
-                      const int m = g + 8 * nt;
-                      uint32_t bf[2] = {0u, 0u};
-                      if (m < M) {
-                        const uint2 v = lds64(xs_addr + ((uint32_t(sl) * M + m) * 16 + t * 4) * 2);
-                        bf[0] = v.x;
-                        bf[1] = v.y;
-                      }
-                      mma_bf16_16816(c[h][nt], a, bf);
-                    }
-                  }
-                } else {
-                  uint32_t ua[2], ub[2];
-                  unpack_u8(wa[wi], ua);
-                  unpack_u8(wb[wi], ub);
-                  const uint32_t a[4] = {ua[0], ub[0], ua[1], ub[1]};
-                  const int sl = slot_base + wi;
+                  const uint32_t a0[4] = {ua[0], ub[0], ua[1], ub[1]};
+                  const uint32_t a1[4] = {ua[2], ub[2], ua[3], ub[3]};
 #pragma unroll
                   for (int nt = 0; nt < MT; ++nt) {
-                    const int m = g + 8 * nt;
-                    uint32_t bf[2] = {0u, 0u};
-                    if (m < M) {
-                      const uint2 v = lds64(xs_addr + ((uint32_t(sl) * M + m) * 16 + t * 4) * 2);
-                      bf[0] = v.x;
-                      bf[1] = v.y;
-                    }
-                    mma_bf16_16816(c[wi & 1][nt], a, bf);
+                    uint4 bv = make_uint4(0u, 0u, 0u, 0u);
+                    if (xv[nt]) bv = lds128(xb[nt] + chunk_off + wi * 64);
+                    const uint32_t b0[2] = {bv.x, bv.y};
+                    const uint32_t b1[2] = {bv.z, bv.w};
+                    mma_bf16_16816(c[0][nt], a0, b0);
+                    mma_bf16_16816(c[1][nt], a1, b1);
+                  }
+                }
+              } else {
+#pragma unroll
+                for (int wi = 0; wi < Geo::kWords; wi += 2) {
+                  uint32_t ua0[2], ub0[2], ua1[2], ub1[2];
+                  unpack_u8(wa[wi], ua0);
+                  unpack_u8(wb[wi], ub0);
+                  unpack_u8(wa[wi + 1], ua1);
+                  unpack_u8(wb[wi + 1], ub1);
+                  const uint32_t a0[4] = {ua0[0], ub0[0], ua0[1], ub0[1]};
+                  const uint32_t a1[4] = {ua1[0], ub1[0], ua1[1], ub1[1]};
+#pragma unroll
+                  for (int nt = 0; nt < MT; ++nt) {
+                    uint4 bv = make_uint4(0u, 0u, 0u, 0u);
+                    if (xv[nt]) bv = lds128(xb[nt] + chunk_off + (wi / 2) * 64);
+                    const uint32_t b0[2] = {bv.x, bv.y};
+                    const uint32_t b1[2] = {bv.z, bv.w};
+                    mma_bf16_16816(c[0][nt], a0, b0);
+                    mma_bf16_16816(c[1][nt], a1, b1);
                   }
                 }
               }
@@ -450,21 +464,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
 
-      // Reduce the SKW partial sums of each row tile in a fixed order.
-      const int per_tile = kBoxRows * M;
+      // Add the SKW partial sums of each row tile in a fixed order.  The
+      // partials go to one of two buffers, so a single barrier per item
+      // suffices: a buffer is rewritten two items later, after another
+      // barrier that every reducer of this item has passed.
+      float* rb = red + (p.red_bufs == 2 ? (local_item & 1) : 0) * red_stride;
 #pragma unroll
       for (int nt = 0; nt < MT; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int m = 8 * nt + 2 * t + (e & 1);
           const int r = g + 8 * (e >> 1);
-          if (m < M) red[(rt * p.SKW + sk) * per_tile + r * M + m] = y[nt][e];
+          if (m < M) rb[(rt * p.SKW + sk) * per_tile + r * M + m] = y[nt][e];
         }
       named_barrier_sync(1, nthr);
-      for (int o = tid; o < p.RT * per_tile; o += nthr) {
+      // rotate which threads reduce, so the work spreads over the warps
+      const int rot = (local_item * 32 * 5) % nthr;
+      const int me = (tid + nthr - rot) % nthr;
+      for (int o = me; o < p.RT * per_tile; o += nthr) {
         const int rto = o / per_tile, rem = o % per_tile;
-        float sum = 0.f;
-        for (int s2 = 0; s2 < p.SKW; ++s2) sum += red[(rto * p.SKW + s2) * per_tile + rem];
+        const float* src = rb + rto * p.SKW * per_tile + rem;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        int s2 = 0;
+        for (; s2 + 4 <= p.SKW; s2 += 4) {
+          acc[0] += src[(s2 + 0) * per_tile];
+          acc[1] += src[(s2 + 1) * per_tile];
+          acc[2] += src[(s2 + 2) * per_tile];
+          acc[3] += src[(s2 + 3) * per_tile];
+        }
+        for (; s2 < p.SKW; ++s2) acc[0] += src[s2 * per_tile];
+        const float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
         if (csize == 1) {
           const int row = (item * p.RT + rto) * kBoxRows + rem / M;
           const int m = rem % M;
@@ -478,8 +507,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           part[size_t(local_item) * p.RT * per_tile + o] = sum;
         }
       }
-      named_barrier_sync(1, nthr);
+      if (p.red_bufs == 1) named_barrier_sync(1, nthr);  // buffer reused by the next item
     }
+    // the last item's reducers must finish before the cluster exchange
+    named_barrier_sync(1, nthr);
   }
 
   if (csize > 1) {

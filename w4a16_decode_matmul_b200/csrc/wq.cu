@@ -153,7 +153,8 @@ const void* gemv_kernel_ptr() {
 // cluster ranks and `bpw` boxes per warp and stage.  False if it does not fit
 // with at least `min_depth` ring stages.
 bool plan_gemv_with(int M, int N, int K, int bits, int group, const DeviceInfo& dev,
-                    int cluster_cap, int C, int bpw, int min_depth, GemvPlan* plan) {
+                    int cluster_cap, int C, int bpw, int min_depth, int red_bufs,
+                    GemvPlan* plan) {
   auto round_up = [](int a, int b) { return (a + b - 1) / b * b; };
   const int box_k = wq::gemv::kBoxRowBytes * 8 / bits;
   const int granule = std::max(box_k, group);
@@ -186,7 +187,10 @@ bool plan_gemv_with(int M, int N, int K, int bits, int group, const DeviceInfo& 
   p.stages_per_item = (kc + stage_k - 1) / stage_k;
   p.meta_tma = (ngroups % 8 == 0 && sg % 8 == 0 && (kc / group) % 8 == 0) ? 1 : 0;
 
-  const uint32_t codes_bytes = uint32_t(RT * skw * bpw * wq::gemv::kBoxBytes);
+  // rows of a stage: stage_k*bits/8 bytes, padded to an odd multiple of 64
+  const uint32_t seg = uint32_t(stage_k * bits / 8);
+  p.row_stride = seg + ((seg / 64) % 2 == 0 ? 64u : 0u);
+  const uint32_t codes_bytes = uint32_t(round_up(int(RT * 16 * p.row_stride), 128));
   const uint32_t meta_bytes = uint32_t(2 * RT * 16 * sg * 2);  // scales + zeros
   p.meta_offset = codes_bytes;
   p.stage_bytes = uint32_t(round_up(int(codes_bytes + meta_bytes), 1024));
@@ -195,9 +199,13 @@ bool plan_gemv_with(int M, int N, int K, int bits, int group, const DeviceInfo& 
   if (cluster_cap > 0) clusters = std::min(clusters, cluster_cap);
   const int items_per_cluster_max = (p.items + clusters - 1) / clusters;
   const size_t off = 1024;  // barriers + flags
-  const size_t fixed_x = size_t(round_up(kc * M * 2, 128));
+  // activation rows: 2*kc bytes padded to an odd multiple of 64 B so that
+  // rows m and m+1 fall in different shared-memory bank halves
+  p.x_row_stride = uint32_t(2 * kc + (((2 * kc) / 64) % 2 == 0 ? 64 : 0));
+  const size_t fixed_x = size_t(round_up(int(p.x_row_stride) * M, 128));
   const size_t fixed_sx = size_t(round_up((kc / group) * 8 * MT * 4, 128));
-  const size_t fixed_red = size_t(round_up(16 * 16 * M * 4, 128));
+  p.red_bufs = red_bufs;
+  const size_t fixed_red = size_t(round_up(red_bufs * 16 * 16 * M * 4, 128));
   const size_t fixed_part =
       C > 1 ? size_t(round_up(items_per_cluster_max * RT * 16 * M * 4, 128)) : 0;
   const size_t fixed = off + fixed_x + fixed_sx + fixed_red + fixed_part;
@@ -221,9 +229,32 @@ bool plan_gemv_with(int M, int N, int K, int bits, int group, const DeviceInfo& 
 // Choose the cluster split and stage size.  K is split across a cluster when
 // there are too few row tiles to fill the SMs, or when the activations would
 // not fit in shared memory; stages shrink before the ring gets shallow.
+// Tuning hook (internal, off by default): force the cluster split, boxes per
+// warp and ring depth of the next plans; 0 keeps the heuristic's choice.
+int g_force_C = 0, g_force_bpw = 0, g_force_depth = 0;
+
 bool plan_gemv(int M, int N, int K, int bits, int group, const DeviceInfo& dev, int cluster_cap,
                GemvPlan* plan) {
   const int tiles = (N + 15) / 16;
+  if (g_force_C > 0 || g_force_bpw > 0) {
+    const int C = g_force_C > 0 ? g_force_C : 1;
+    const int bpw = g_force_bpw > 0 ? g_force_bpw : 1;
+    for (int red_bufs : {2, 1})
+      if (plan_gemv_with(M, N, K, bits, group, dev, cluster_cap, C, bpw, 2, red_bufs, plan)) {
+        if (g_force_depth > 0 && g_force_depth < plan->p.depth) {
+          const int d = g_force_depth;
+          const uint32_t shift = uint32_t(plan->p.depth - d) * plan->p.stage_bytes;
+          plan->p.depth = d;
+          plan->p.off_x -= shift;
+          plan->p.off_sx -= shift;
+          plan->p.off_red -= shift;
+          plan->p.off_part -= shift;
+          plan->smem -= shift;
+        }
+        return true;
+      }
+    return false;
+  }
   const int sms = dev.sms;
   int C0 = 1;
   if (tiles < 3 * sms) C0 = 2;
@@ -232,14 +263,17 @@ bool plan_gemv(int M, int N, int K, int bits, int group, const DeviceInfo& dev, 
   const int bpw_min = (bits == 8 && group == 128) ? 2 : 1;
   const int bpw_max = bits == 8 ? 4 : 2;
   for (int min_depth : {3, 2}) {
-    for (int C = C0; C <= 16; C *= 2) {
-      const int box_k = wq::gemv::kBoxRowBytes * 8 / bits;
-      const int granule = std::max(box_k, group);
-      const int kc = (((K + C - 1) / C) + granule - 1) / granule * granule;
-      if (size_t(kc) * M * 2 > 128 * 1024 && C < 16) continue;
-      for (int bpw = bpw_max; bpw >= bpw_min; bpw /= 2)
-        if (plan_gemv_with(M, N, K, bits, group, dev, cluster_cap, C, bpw, min_depth, plan))
-          return true;
+    for (int red_bufs : {2, 1}) {
+      for (int C = C0; C <= 16; C *= 2) {
+        const int box_k = wq::gemv::kBoxRowBytes * 8 / bits;
+        const int granule = std::max(box_k, group);
+        const int kc = (((K + C - 1) / C) + granule - 1) / granule * granule;
+        if (size_t(kc) * M * 2 > 128 * 1024 && C < 16) continue;
+        for (int bpw = bpw_max; bpw >= bpw_min; bpw /= 2)
+          if (plan_gemv_with(M, N, K, bits, group, dev, cluster_cap, C, bpw, min_depth, red_bufs,
+                             plan))
+            return true;
+      }
     }
   }
   return false;
@@ -288,6 +322,7 @@ cudaError_t launch_gemv_t(GemvPlan& plan, const DeviceInfo& dev, const void* cod
       plan.p.Y = keep.Y;
       plan.p.scales = keep.scales;
       plan.p.zeros = keep.zeros;
+      plan.p.codes = keep.codes;
       plan.p.y_bf16 = keep.y_bf16;
     }
   }
@@ -401,6 +436,7 @@ wq_status wq_matmul(const void* X, int64_t M, const void* codes, const void* sca
   plan.p.Y = Y;
   plan.p.scales = static_cast<const __half*>(scales);
   plan.p.zeros = static_cast<const __half*>(zeros);
+  plan.p.codes = static_cast<const uint8_t*>(codes);
   plan.p.y_bf16 = out_dtype == WQ_OUT_BF16;
   const cudaError_t e = dispatch_format<GemvOp>(bits, symmetric != 0, group, &plan, &dev, codes,
                                                 scales, zeros,
@@ -432,9 +468,16 @@ const char* wq_status_string(wq_status status) {
 
 const char* wq_version(void) { return "wq 0.1.0 (sm_100a)"; }
 
+// Tuning hook, not part of the public ABI (see g_force_C).
+void wq_internal_force_gemv_plan(int C, int bpw, int depth) {
+  g_force_C = C;
+  g_force_bpw = bpw;
+  g_force_depth = depth;
+}
+
 // Test hook, not part of the public ABI: the matmul plan for a device with
 // `sms` SMs and `smem_optin` bytes of shared memory per block, written to
-// out[0..23] (see tests/test_plan.py for the field order).  Returns 0 if no
+// out[0..26] (see tests/test_plan.py for the field order).  Returns 0 if no
 // plan exists.
 int wq_internal_plan_gemv(int M, int N, int K, int bits, int group, int sms, int smem_optin,
                           int cluster_cap, int64_t* out) {
@@ -448,7 +491,8 @@ int wq_internal_plan_gemv(int M, int N, int K, int bits, int group, int sms, int
                        p.items,   p.RT,          p.SKW,       p.BPW,         p.depth,
                        p.kc,      p.stage_k,     p.stages_per_item, p.meta_tma, p.stage_bytes,
                        p.meta_offset, p.off_ring, p.off_x,    p.off_sx,      p.off_red,
-                       p.off_part, int64_t(plan.smem), plan.C, plan.grid};
+                       p.off_part, int64_t(plan.smem), plan.C, plan.grid, p.x_row_stride,
+                       p.red_bufs, p.row_stride};
   for (size_t i = 0; i < sizeof(v) / sizeof(v[0]); ++i) out[i] = v[i];
   return 1;
 }
