@@ -16,7 +16,7 @@ LIB = os.path.join(ROOT, "w4a16_decode_matmul_b200", "libwq.so")
 FIELDS = ["M", "N", "K", "ngroups", "row_tiles", "items", "RT", "SKW", "BPW", "depth", "kc",
           "stage_k", "stages_per_item", "meta_tma", "stage_bytes", "meta_offset", "off_ring",
           "off_x", "off_sx", "off_red", "off_part", "smem", "C", "grid", "x_row_stride",
-          "red_bufs", "row_stride"]
+          "red_bufs", "row_stride", "contig"]
 B200_SMS = 148
 B200_SMEM_OPTIN = 232448
 
@@ -62,7 +62,11 @@ def check_plan(p, bits, G):
     assert p["stage_k"] % G == 0
     rs = p["row_stride"]
     seg_max = p["stage_k"] * bits // 8
-    assert rs % 16 == 0 and rs >= seg_max and rs % 128 == 64     # odd multiple of 64
+    assert rs % 16 == 0 and rs >= seg_max and rs % 64 == 0     # padded to an odd multiple of 64 when it fits
+    if p["contig"]:
+        # whole rows arrive by single copies: dense rows, all groups' metadata
+        assert C == 1 and p["stage_k"] == K and rs == seg_max and p["meta_tma"]
+        assert sg == p["ngroups"] and 16 * p["ngroups"] * 2 % 16 == 0
     codes_bytes = p["RT"] * 16 * rs
     meta_rt = 16 * sg * 2
     assert p["meta_offset"] >= codes_bytes and p["meta_offset"] % 128 == 0
@@ -71,14 +75,15 @@ def check_plan(p, bits, G):
     assert p["meta_offset"] + 2 * p["RT"] * meta_rt <= p["stage_bytes"]
     assert p["off_ring"] + p["depth"] * p["stage_bytes"] <= p["off_x"]
     xrow = p["x_row_stride"]
-    assert xrow % 64 == 0 and (xrow // 64) % 2 == 1 and xrow >= 2 * p["kc"]
-    assert p["off_x"] + xrow * M <= p["off_sx"]
+    assert xrow % 64 == 0 and xrow >= 2 * p["kc"]
+    assert p["off_x"] + xrow * (M + 1) <= p["off_sx"]      # + the zero row
     assert p["off_sx"] + (p["kc"] // G) * 8 * MT * 4 <= p["off_red"]
-    assert p["red_bufs"] in (1, 2)
-    assert p["off_red"] + p["red_bufs"] * 16 * 16 * M * 4 <= p["off_part"]
     clusters = p["grid"] // C
     assert p["grid"] % C == 0 and clusters >= 1 and C <= 16
     per_cluster = -(-p["items"] // clusters)
+    assert p["red_bufs"] in (0, 1, 2)
+    red_slots = per_cluster if p["red_bufs"] == 0 else p["red_bufs"]
+    assert p["off_red"] + red_slots * 16 * 16 * M * 4 <= p["off_part"]
     if C > 1:
         assert p["off_part"] + per_cluster * p["RT"] * 16 * M * 4 <= p["smem"]
     assert p["kc"] % max(geo["box_k"], G) == 0
@@ -165,17 +170,8 @@ CASES = (
 )
 
 
-# Small-batch shapes whose shared-memory footprint has no plan yet; the
-# library returns WQ_ERR_UNSUPPORTED for them.
-NO_PLAN = {(32, 4096, 14336, 8, 128)}
-
-
 @pytest.mark.parametrize("M,N,K,bits,G", CASES)
 def test_plan_and_indices(lib, M, N, K, bits, G):
-    if (M, N, K, bits, G) in NO_PLAN:
-        out = (ctypes.c_int64 * 32)()
-        assert lib.wq_internal_plan_gemv(M, N, K, bits, G, B200_SMS, B200_SMEM_OPTIN, 0, out) == 0
-        return
     check_plan(plan(lib, M, N, K, bits, G), bits, G)
 
 

@@ -144,16 +144,11 @@ struct GemvPlan {
   size_t smem = 0;
 };
 
-template <int BITS, bool SYM, int G, int MT>
-const void* gemv_kernel_ptr() {
-  return reinterpret_cast<const void*>(&wq::gemv::gemv_kernel<BITS, SYM, G, MT>);
-}
-
 // Shared-memory layout and work split for one call with K split over C
 // cluster ranks and `bpw` boxes per warp and stage.  False if it does not fit
 // with at least `min_depth` ring stages.
 bool plan_gemv_with(int M, int N, int K, int bits, int group, const DeviceInfo& dev,
-                    int cluster_cap, int C, int bpw, int min_depth, int red_bufs,
+                    int cluster_cap, int C, int bpw, int min_depth, int red_bufs, bool pad,
                     GemvPlan* plan) {
   auto round_up = [](int a, int b) { return (a + b - 1) / b * b; };
   const int box_k = wq::gemv::kBoxRowBytes * 8 / bits;
@@ -187,25 +182,30 @@ bool plan_gemv_with(int M, int N, int K, int bits, int group, const DeviceInfo& 
   p.stages_per_item = (kc + stage_k - 1) / stage_k;
   p.meta_tma = (ngroups % 8 == 0 && sg % 8 == 0 && (kc / group) % 8 == 0) ? 1 : 0;
 
-  // rows of a stage: stage_k*bits/8 bytes, padded to an odd multiple of 64
+  // rows of a stage: stage_k*bits/8 bytes, padded to an odd multiple of 64;
+  // whole-row stages (one cluster rank, one stage of all K) stay dense so the
+  // item arrives by single bulk copies
   const uint32_t seg = uint32_t(stage_k * bits / 8);
-  p.row_stride = seg + ((seg / 64) % 2 == 0 ? 64u : 0u);
+  p.contig = (C == 1 && stage_k == K && p.meta_tma) ? 1 : 0;
+  p.row_stride = seg + (pad && !p.contig && (seg / 64) % 2 == 0 ? 64u : 0u);
   const uint32_t codes_bytes = uint32_t(round_up(int(RT * 16 * p.row_stride), 128));
   const uint32_t meta_bytes = uint32_t(2 * RT * 16 * sg * 2);  // scales + zeros
   p.meta_offset = codes_bytes;
   p.stage_bytes = uint32_t(round_up(int(codes_bytes + meta_bytes), 1024));
 
+  const size_t off = 1024;  // barriers + flags
   int clusters = std::max(1, dev.sms / C);
   if (cluster_cap > 0) clusters = std::min(clusters, cluster_cap);
   const int items_per_cluster_max = (p.items + clusters - 1) / clusters;
-  const size_t off = 1024;  // barriers + flags
   // activation rows: 2*kc bytes padded to an odd multiple of 64 B so that
   // rows m and m+1 fall in different shared-memory bank halves
-  p.x_row_stride = uint32_t(2 * kc + (((2 * kc) / 64) % 2 == 0 ? 64 : 0));
-  const size_t fixed_x = size_t(round_up(int(p.x_row_stride) * M, 128));
+  p.x_row_stride = uint32_t(2 * kc + (pad && ((2 * kc) / 64) % 2 == 0 ? 64 : 0));
+  const size_t fixed_x = size_t(round_up(int(p.x_row_stride) * (M + 1), 128));  // + a zero row
   const size_t fixed_sx = size_t(round_up((kc / group) * 8 * MT * 4, 128));
+  // red_bufs == 0: one partial-sum slot per item of the CTA (no per-item barrier)
   p.red_bufs = red_bufs;
-  const size_t fixed_red = size_t(round_up(red_bufs * 16 * 16 * M * 4, 128));
+  const int red_slots = red_bufs == 0 ? items_per_cluster_max : red_bufs;
+  const size_t fixed_red = size_t(round_up(red_slots * 16 * 16 * M * 4, 128));
   const size_t fixed_part =
       C > 1 ? size_t(round_up(items_per_cluster_max * RT * 16 * M * 4, 128)) : 0;
   const size_t fixed = off + fixed_x + fixed_sx + fixed_red + fixed_part;
@@ -240,7 +240,7 @@ bool plan_gemv(int M, int N, int K, int bits, int group, const DeviceInfo& dev, 
     const int C = g_force_C > 0 ? g_force_C : 1;
     const int bpw = g_force_bpw > 0 ? g_force_bpw : 1;
     for (int red_bufs : {2, 1})
-      if (plan_gemv_with(M, N, K, bits, group, dev, cluster_cap, C, bpw, 2, red_bufs, plan)) {
+      if (plan_gemv_with(M, N, K, bits, group, dev, cluster_cap, C, bpw, 2, red_bufs, true, plan)) {
         if (g_force_depth > 0 && g_force_depth < plan->p.depth) {
           const int d = g_force_depth;
           const uint32_t shift = uint32_t(plan->p.depth - d) * plan->p.stage_bytes;
@@ -263,26 +263,27 @@ bool plan_gemv(int M, int N, int K, int bits, int group, const DeviceInfo& dev, 
   const int bpw_min = (bits == 8 && group == 128) ? 2 : 1;
   const int bpw_max = bits == 8 ? 4 : 2;
   for (int min_depth : {3, 2}) {
-    for (int red_bufs : {2, 1}) {
+    for (int red_bufs : {0, 2, 1}) {
       for (int C = C0; C <= 16; C *= 2) {
         const int box_k = wq::gemv::kBoxRowBytes * 8 / bits;
         const int granule = std::max(box_k, group);
         const int kc = (((K + C - 1) / C) + granule - 1) / granule * granule;
         if (size_t(kc) * M * 2 > 128 * 1024 && C < 16) continue;
         for (int bpw = bpw_max; bpw >= bpw_min; bpw /= 2)
-          if (plan_gemv_with(M, N, K, bits, group, dev, cluster_cap, C, bpw, min_depth, red_bufs,
-                             plan))
-            return true;
+          for (bool pad : {true, false})  // unpadded rows (bank conflicts) only as a last resort
+            if (plan_gemv_with(M, N, K, bits, group, dev, cluster_cap, C, bpw, min_depth, red_bufs,
+                               pad, plan))
+              return true;
       }
     }
   }
   return false;
 }
 
-template <int BITS, bool SYM, int G, int MT>
+template <int BITS, bool SYM, int G, int MT, int MEFF, bool FAST>
 cudaError_t launch_gemv_t(GemvPlan& plan, const DeviceInfo& dev, const void* codes,
                           const void* scales, const void* zeros, cudaStream_t s) {
-  auto kernel = &wq::gemv::gemv_kernel<BITS, SYM, G, MT>;
+  auto kernel = &wq::gemv::gemv_kernel<BITS, SYM, G, MT, MEFF, FAST>;
   static int configured_smem[kMaxDevices] = {};  // per instantiation and device
   int device = 0;
   cudaGetDevice(&device);
@@ -353,10 +354,23 @@ template <int BITS, bool SYM, int G>
 struct GemvOp {
   static cudaError_t run(GemvPlan* plan, const DeviceInfo* dev, const void* c, const void* sc,
                          const void* z, cudaStream_t s) {
+    // M <= 8: one n8 tile whose columns hold up to 8/MEFF groups of MEFF rows
     const int M = plan->p.M;
-    if (M <= 8) return launch_gemv_t<BITS, SYM, G, 1>(*plan, *dev, c, sc, z, s);
-    if (M <= 16) return launch_gemv_t<BITS, SYM, G, 2>(*plan, *dev, c, sc, z, s);
-    return launch_gemv_t<BITS, SYM, G, 4>(*plan, *dev, c, sc, z, s);
+    // the unrolled path: one stage per item with the format's natural box count
+    const bool fast = M <= 8 && plan->p.stages_per_item == 1 &&
+                      plan->p.BPW == wq::gemv::FastShape<BITS>::kBPW;
+    if (fast) {
+      if (M == 1) return launch_gemv_t<BITS, SYM, G, 1, 1, true>(*plan, *dev, c, sc, z, s);
+      if (M == 2) return launch_gemv_t<BITS, SYM, G, 1, 2, true>(*plan, *dev, c, sc, z, s);
+      if (M <= 4) return launch_gemv_t<BITS, SYM, G, 1, 4, true>(*plan, *dev, c, sc, z, s);
+      return launch_gemv_t<BITS, SYM, G, 1, 8, true>(*plan, *dev, c, sc, z, s);
+    }
+    if (M == 1) return launch_gemv_t<BITS, SYM, G, 1, 1, false>(*plan, *dev, c, sc, z, s);
+    if (M == 2) return launch_gemv_t<BITS, SYM, G, 1, 2, false>(*plan, *dev, c, sc, z, s);
+    if (M <= 4) return launch_gemv_t<BITS, SYM, G, 1, 4, false>(*plan, *dev, c, sc, z, s);
+    if (M <= 8) return launch_gemv_t<BITS, SYM, G, 1, 8, false>(*plan, *dev, c, sc, z, s);
+    if (M <= 16) return launch_gemv_t<BITS, SYM, G, 2, 8, false>(*plan, *dev, c, sc, z, s);
+    return launch_gemv_t<BITS, SYM, G, 4, 8, false>(*plan, *dev, c, sc, z, s);
   }
 };
 
@@ -477,7 +491,7 @@ void wq_internal_force_gemv_plan(int C, int bpw, int depth) {
 
 // Test hook, not part of the public ABI: the matmul plan for a device with
 // `sms` SMs and `smem_optin` bytes of shared memory per block, written to
-// out[0..26] (see tests/test_plan.py for the field order).  Returns 0 if no
+// out[0..27] (see tests/test_plan.py for the field order).  Returns 0 if no
 // plan exists.
 int wq_internal_plan_gemv(int M, int N, int K, int bits, int group, int sms, int smem_optin,
                           int cluster_cap, int64_t* out) {
@@ -492,7 +506,7 @@ int wq_internal_plan_gemv(int M, int N, int K, int bits, int group, int sms, int
                        p.kc,      p.stage_k,     p.stages_per_item, p.meta_tma, p.stage_bytes,
                        p.meta_offset, p.off_ring, p.off_x,    p.off_sx,      p.off_red,
                        p.off_part, int64_t(plan.smem), plan.C, plan.grid, p.x_row_stride,
-                       p.red_bufs, p.row_stride};
+                       p.red_bufs, p.row_stride, p.contig};
   for (size_t i = 0; i < sizeof(v) / sizeof(v[0]); ++i) out[i] = v[i];
   return 1;
 }
