@@ -43,7 +43,7 @@ WORKLOAD = ("decode GEMV, Llama-8B gate/up layer: M=1, K=4096, N=14336, INT4 asy
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "gemv_w4a16_m1_k4096_n14336.json")
 KERNEL_SOURCES = [os.path.join(ROOT, "w4a16_decode_matmul_b200", "csrc", f)
-                  for f in ("gemv.cuh", "common.cuh")]
+                  for f in ("gemv.cuh", "common.cuh", "wq.cu")]
 
 
 def algorithmic_bytes(m: int = M, n: int = N, k: int = K, bits: int = BITS,
