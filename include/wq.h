@@ -108,16 +108,45 @@ wq_status wq_dequantize(const void *codes, const void *scales, const void *zeros
                         int64_t N, int64_t K, int bits, int group, int symmetric,
                         void *W_out, wq_stream_t stream);
 
+/* Flags of wq_matmul. */
+enum {
+    /* The weights (codes, scales, zeros) are not written by the kernel that
+     * precedes this call on `stream`.  The call may then be launched as a
+     * programmatic dependent of that kernel: it starts streaming the weights
+     * while the previous kernel finishes, and reads X, writes Y and touches
+     * the workspace only after the previous kernel has completed.  Use it for
+     * the static weights of a model's layers, not right after wq_quantize of
+     * the same weights. */
+    WQ_MATMUL_STATIC_WEIGHTS = 1
+};
+
+/* Bytes of the matmul workspace (a device buffer, 16-byte aligned, filled
+ * with zeros by the caller before its first use; every completed call leaves
+ * it filled with zeros again). */
+size_t wq_matmul_workspace_bytes(void);
+
 /* Y [M][N] = X [M][K] * What^T, weights formed on chip from codes, scales
  * and zeros and never written to memory.  out_dtype is WQ_OUT_F32 or
  * WQ_OUT_BF16 (round-to-nearest-even from the binary32 accumulator).
- * M <= 32 runs the small-batch decode kernel (codes streamed once from HBM,
+ * M <= 32 runs the small-batch decode kernels (codes streamed once from HBM,
  * tensor-core products of integer-valued bfloat16 codes, binary32 group
- * scaling); larger M runs the prefill kernel.  Deterministic: the same
- * inputs give the same bits on every call. */
+ * scaling); M > 32 returns WQ_ERR_UNSUPPORTED in this build.
+ *
+ * workspace / workspace_bytes: NULL and 0, or a buffer of at least
+ * wq_matmul_workspace_bytes() bytes as described there.  With it, every SM
+ * streams the same number of bytes (row tiles may be summed across CTAs
+ * through the workspace, in a fixed order); without it, whole row tiles are
+ * divided among the SMs.  Calls that may run at the same time on the GPU
+ * (different streams) need different workspaces.  After a call that recorded
+ * WQ_ERR_TIMEOUT the workspace must be zero-filled again.
+ *
+ * flags: 0 or WQ_MATMUL_STATIC_WEIGHTS.
+ *
+ * Deterministic: the same inputs give the same bits on every call. */
 wq_status wq_matmul(const void *X, int64_t M, const void *codes, const void *scales,
                     const void *zeros, int64_t N, int64_t K, int bits, int group,
-                    int symmetric, void *Y, int out_dtype, wq_stream_t stream);
+                    int symmetric, void *Y, int out_dtype, void *workspace,
+                    size_t workspace_bytes, unsigned int flags, wq_stream_t stream);
 
 /* Read and clear the device status word (WQ_OK if no kernel recorded an
  * error).  Synchronizes `stream` first. */

@@ -93,15 +93,27 @@ def test_matmul_rejects_bad_arguments_before_launch(lib):
     f = lib.wq_matmul
     f.restype = ctypes.c_int
     i64, i32, vp = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p
-    f.argtypes = [vp, i64, vp, vp, vp, i64, i64, i32, i32, i32, vp, i32, vp]
+    sz, u32 = ctypes.c_size_t, ctypes.c_uint
+    f.argtypes = [vp, i64, vp, vp, vp, i64, i64, i32, i32, i32, vp, i32, vp, sz, u32, vp]
     p = ctypes.c_void_p(1 << 20)
     bad = ctypes.c_void_p((1 << 20) + 8)
-    assert f(p, 0, p, p, p, 64, 128, 4, 32, 0, p, 0, None) == 1      # M
-    assert f(p, 1, p, p, p, 64, 128, 4, 32, 0, p, 7, None) == 1      # out dtype
-    assert f(p, 1, p, p, None, 64, 128, 4, 32, 0, p, 0, None) == 1   # zeros missing
-    assert f(p, 1, p, p, p, 64, 120, 4, 32, 0, p, 0, None) == 1      # K
-    assert f(bad, 1, p, p, p, 64, 128, 4, 32, 0, p, 0, None) == 3    # X alignment
-    assert f(p, 1, p, p, p, 64, 128, 4, 32, 0, bad, 0, None) == 3    # Y alignment
+    assert f(p, 0, p, p, p, 64, 128, 4, 32, 0, p, 0, None, 0, 0, None) == 1      # M
+    assert f(p, 1, p, p, p, 64, 128, 4, 32, 0, p, 7, None, 0, 0, None) == 1      # out dtype
+    assert f(p, 1, p, p, None, 64, 128, 4, 32, 0, p, 0, None, 0, 0, None) == 1   # zeros missing
+    assert f(p, 1, p, p, p, 64, 120, 4, 32, 0, p, 0, None, 0, 0, None) == 1      # K
+    assert f(p, 1, p, p, p, 64, 128, 4, 32, 0, p, 0, None, 0, 2, None) == 1      # flags
+    assert f(p, 1, p, p, p, 64, 128, 4, 32, 0, p, 0, None, 64, 0, None) == 1     # bytes, no buffer
+    assert f(bad, 1, p, p, p, 64, 128, 4, 32, 0, p, 0, None, 0, 0, None) == 3    # X alignment
+    assert f(p, 1, p, p, p, 64, 128, 4, 32, 0, bad, 0, None, 0, 0, None) == 3    # Y alignment
+    assert f(p, 1, p, p, p, 64, 128, 4, 32, 0, p, 0, bad, 1 << 20, 0, None) == 3  # workspace
+
+
+def test_workspace_size(lib):
+    f = lib.wq_matmul_workspace_bytes
+    f.restype = ctypes.c_size_t
+    f.argtypes = []
+    # flags for 1024 CTAs + 1024 x 16 rows x 8 activation rows of binary32 partials
+    assert f() == 1024 * 4 + 1024 * 128 * 4
 
 
 def test_dequantize_rejects_bad_arguments_before_launch(lib):

@@ -2,8 +2,8 @@
 
 Argument marshalling only: every step of quantize, dequantize and matmul
 runs in the library's CUDA kernels.  PyTorch provides device memory and the
-current stream.  The library must have been built (``python -m
-w4a16_decode_matmul_b200.build``); importing this package without it raises.
+current stream.  The library must have been built (``python
+w4a16_decode_matmul_b200/build.py``); importing this package without it raises.
 
 Functions keep the C names without the ``wq_`` prefix:
 
@@ -27,6 +27,7 @@ LIBRARY_PATH = os.path.join(_HERE, "libwq.so")
 WQ_OK = 0
 WQ_OUT_F32 = 0
 WQ_OUT_BF16 = 1
+WQ_MATMUL_STATIC_WEIGHTS = 1
 
 STATUS_NAMES = {0: "WQ_OK", 1: "WQ_ERR_INVALID_ARG", 2: "WQ_ERR_UNSUPPORTED",
                 3: "WQ_ERR_ALIGNMENT", 4: "WQ_ERR_CUDA", 5: "WQ_ERR_TIMEOUT"}
@@ -35,13 +36,16 @@ STATUS_NAMES = {0: "WQ_OK", 1: "WQ_ERR_INVALID_ARG", 2: "WQ_ERR_UNSUPPORTED",
 class WQError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
-        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)} ({status_string(status)})")
+        detail = status_string(status)
+        if status == 4:
+            detail += ": " + lib.wq_internal_last_cuda_error().decode()
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)} ({detail})")
 
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIBRARY_PATH):
         raise ImportError(
-            f"{LIBRARY_PATH} is missing: build it with `python -m w4a16_decode_matmul_b200.build`")
+            f"{LIBRARY_PATH} is missing: build it with `python w4a16_decode_matmul_b200/build.py`")
     lib = ctypes.CDLL(LIBRARY_PATH)
     i64, i32, vp, sz = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
     lib.wq_codes_bytes.argtypes = [i64, i64, i32]
@@ -52,7 +56,10 @@ def _load() -> ctypes.CDLL:
     lib.wq_quantize.restype = i32
     lib.wq_dequantize.argtypes = [vp, vp, vp, i64, i64, i32, i32, i32, vp, vp]
     lib.wq_dequantize.restype = i32
-    lib.wq_matmul.argtypes = [vp, i64, vp, vp, vp, i64, i64, i32, i32, i32, vp, i32, vp]
+    lib.wq_matmul_workspace_bytes.argtypes = []
+    lib.wq_matmul_workspace_bytes.restype = sz
+    lib.wq_matmul.argtypes = [vp, i64, vp, vp, vp, i64, i64, i32, i32, i32, vp, i32, vp, sz,
+                              ctypes.c_uint, vp]
     lib.wq_matmul.restype = i32
     lib.wq_get_device_error.argtypes = [vp]
     lib.wq_get_device_error.restype = i32
@@ -60,6 +67,8 @@ def _load() -> ctypes.CDLL:
     lib.wq_status_string.restype = ctypes.c_char_p
     lib.wq_version.argtypes = []
     lib.wq_version.restype = ctypes.c_char_p
+    lib.wq_internal_last_cuda_error.argtypes = []
+    lib.wq_internal_last_cuda_error.restype = ctypes.c_char_p
     return lib
 
 
@@ -158,13 +167,32 @@ def dequantize(qw: QuantizedWeight, out: torch.Tensor | None = None) -> torch.Te
     return out
 
 
+_workspaces: dict = {}
+
+
+def workspace(device: torch.device, stream: int) -> torch.Tensor:
+    """The zero-filled ``wq_matmul`` workspace used for calls on ``stream``
+    (one per device and stream, so that calls on different streams never
+    share one)."""
+    key = (device.index, stream)
+    ws = _workspaces.get(key)
+    if ws is None:
+        ws = torch.zeros(lib.wq_matmul_workspace_bytes(), dtype=torch.uint8, device=device)
+        _workspaces[key] = ws
+    return ws
+
+
 def matmul(X: torch.Tensor, qw: QuantizedWeight, out_dtype: torch.dtype = torch.float32,
-           out: torch.Tensor | None = None) -> torch.Tensor:
+           out: torch.Tensor | None = None, static_weights: bool = False,
+           use_workspace: bool = True) -> torch.Tensor:
     """``wq_matmul``: Y [M, N] = X [M, K] (bfloat16) times What^T.
 
     X may live on the host: it is then copied to the weights' device, the
     product is computed there and Y is copied back to the host (the
-    end-to-end path; pinned host memory makes the copies asynchronous)."""
+    end-to-end path; pinned host memory makes the copies asynchronous).
+    ``static_weights`` passes WQ_MATMUL_STATIC_WEIGHTS: the weights are not
+    written by the kernel that precedes the call on the stream.
+    ``use_workspace=False`` passes no workspace (whole row tiles per SM)."""
     if X.dtype != torch.bfloat16 or X.dim() != 2 or X.shape[1] != qw.K:
         raise ValueError("X must be a 2-D bfloat16 tensor [M, K]")
     if out_dtype not in (torch.float32, torch.bfloat16):
@@ -177,10 +205,14 @@ def matmul(X: torch.Tensor, qw: QuantizedWeight, out_dtype: torch.dtype = torch.
     Yd = out if (out is not None and out.is_cuda) else torch.empty(
         (M, qw.N), dtype=out_dtype, device=dev)
     _require_cuda(Yd)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    ws = workspace(dev, stream) if use_workspace else None
     _check(lib.wq_matmul(_ptr(Xd), M, _ptr(qw.codes), _ptr(qw.scales), _ptr(qw.zeros), qw.N,
                          qw.K, qw.bits, qw.group, int(qw.symmetric), _ptr(Yd),
                          WQ_OUT_BF16 if Yd.dtype == torch.bfloat16 else WQ_OUT_F32,
-                         _stream(dev)), "wq_matmul")
+                         _ptr(ws), 0 if ws is None else ws.numel(),
+                         WQ_MATMUL_STATIC_WEIGHTS if static_weights else 0,
+                         ctypes.c_void_p(stream)), "wq_matmul")
     if not host:
         return Yd
     if out is not None and not out.is_cuda:

@@ -1,6 +1,8 @@
 """Build the CUDA library ``libwq.so`` in-tree for sm_100a.
 
-    python -m w4a16_decode_matmul_b200.build [--force]
+    python w4a16_decode_matmul_b200/build.py [--force]
+
+(run as a script: importing the package loads the library it builds)
 """
 from __future__ import annotations
 

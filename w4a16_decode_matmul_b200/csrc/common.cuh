@@ -18,6 +18,7 @@ __device__ unsigned int g_status;
 // A wait gives up after this many nanoseconds of wall time (globaltimer).
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 constexpr unsigned int kStatusTimeout = 5;                  // WQ_ERR_TIMEOUT
+constexpr unsigned int kStatusInternal = 4;                 // WQ_ERR_CUDA: inconsistent launch
 
 __device__ __forceinline__ void record_status(unsigned int code) {
   atomicCAS(&g_status, 0u, code);
@@ -82,6 +83,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// As mbar_wait, for a thread with nothing else to do: sleeps between polls
+// so that it does not take issue slots from the warps that share its SM
+// sub-partition.
+__device__ __forceinline__ bool mbar_wait_idle(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long start = global_timer_ns();
+  while (true) {
+    __nanosleep(64);
+    if (mbar_try_wait(bar, parity)) return true;
+    if (global_timer_ns() - start > kWaitLimitNs) {
+      record_status(kStatusTimeout);
+      return false;
+    }
+  }
+}
+
 // ---- TMA ------------------------------------------------------------------
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
@@ -96,6 +113,18 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_addr(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+
+// 3-D tile load global -> shared (x innermost).  With a swizzled map the
+// destination must be 1024-byte aligned.
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t x, int32_t y, int32_t z, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(y), "r"(z),
+      "l"(policy)
       : "memory");
 }
 
@@ -126,6 +155,10 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last() {
 
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+__device__ __forceinline__ void named_barrier_arrive(uint32_t id, uint32_t threads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
 // ---- clusters / distributed shared memory ------------------------------------
@@ -203,6 +236,41 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
   uint32_t v;
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
   return v;
+}
+
+// Four 8x8 matrices of 16-bit elements: lane i supplies the address of row
+// i % 8 of matrix i / 8; register j of lane (g, t) receives the 32 bits at
+// byte 4t of row g of matrix j.
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                            uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// ---- flags between CTAs of one grid ---------------------------------------------
+
+__device__ __forceinline__ void st_release_gpu(unsigned int* p, unsigned int v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* p) {
+  unsigned int v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Wait until *flag == 1; false (and the status word set) after kWaitLimitNs.
+__device__ __forceinline__ bool wait_flag(const unsigned int* flag) {
+  if (ld_acquire_gpu(flag) == 1u) return true;
+  const unsigned long long start = global_timer_ns();
+  while (true) {
+    if (ld_acquire_gpu(flag) == 1u) return true;
+    if (global_timer_ns() - start > kWaitLimitNs) {
+      record_status(kStatusTimeout);
+      return false;
+    }
+  }
 }
 
 // ---- streaming global loads ------------------------------------------------------

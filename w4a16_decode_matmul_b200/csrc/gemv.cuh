@@ -40,6 +40,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "unpack.cuh"
 
 namespace wq {
 namespace gemv {
@@ -77,46 +78,6 @@ struct Params {
                            // item's codes and metadata are contiguous and arrive by one
                            // bulk copy each
 };
-
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4],
-                                               const uint32_t (&b)[2]) {
-  // not volatile: a pure function of its registers, free to be scheduled
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
-      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-
-__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t bits) {
-  uint32_t r;
-  // (a & mask) | bits
-  asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(r) : "r"(a), "r"(mask), "r"(bits));
-  return r;
-}
-
-// Eight 4-bit codes of one 32-bit word -> four bfloat16 pairs (128 + u):
-// r[i] = (u_i, u_{i+4}) for i = 0..3 (low half first).
-__device__ __forceinline__ void unpack_u4(uint32_t w, uint32_t (&r)[4]) {
-  constexpr uint32_t kMask = 0x000F000Fu, kMagic = 0x43004300u;  // bf16 128.0 pair
-  r[0] = lop3_and_or(w, kMask, kMagic);
-  r[1] = lop3_and_or(w >> 4, kMask, kMagic);
-  r[2] = lop3_and_or(w >> 8, kMask, kMagic);
-  r[3] = lop3_and_or(w >> 12, kMask, kMagic);
-}
-
-// Four 8-bit codes -> two bfloat16 pairs (u0, u1), (u2, u3), exact integers.
-__device__ __forceinline__ void unpack_u8(uint32_t w, uint32_t (&r)[2]) {
-  float f[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    // 2^23 + u as binary32, minus 2^23: exact
-    f[i] = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7650 | i)) - 8388608.0f;
-  }
-  __nv_bfloat162 p0 = __floats2bfloat162_rn(f[0], f[1]);
-  __nv_bfloat162 p1 = __floats2bfloat162_rn(f[2], f[3]);
-  r[0] = *reinterpret_cast<uint32_t*>(&p0);
-  r[1] = *reinterpret_cast<uint32_t*>(&p1);
-}
 
 // Shared-memory loads as plain C++ accesses (offsets from the dynamic
 // shared-memory base): ordered after the mbarrier waits, whose asm carries a
@@ -198,8 +159,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   __syncthreads();
-
-  grid_dependency_wait();
+  // Kernels launched after this one may be scheduled; they wait for this
+  // grid before touching its outputs.  The weights are read before the wait
+  // for the previous grid (they are not written by it, as the caller
+  // promises when it asks for programmatic dependent launch).
+  grid_dependents_launch();
 
   uint8_t* ring = smem + p.off_ring;
   constexpr bool kAsymMeta = !SYM;
@@ -303,6 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ consumers
+    grid_dependency_wait();  // activations and outputs belong to the previous grid until then
     const int tid = threadIdx.x;  // 0 .. 16*32-1
     const int nthr = kNumConsumerWarps * 32;
     const int M = p.M;

@@ -11,6 +11,7 @@
 #include "common.cuh"
 #include "quantize.cuh"
 #include "gemv.cuh"
+#include "gemv_sk.cuh"
 
 namespace {
 
@@ -68,6 +69,24 @@ bool encode_2d(CUtensorMap* map, const void* base, CUtensorMapDataType type, int
   CUresult r = fn(map, type, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// 3-D view: dims {d0, d1, d2} (d0 innermost, contiguous), byte strides of d1
+// and d2 (any order), box {b0, b1, b2}.
+bool encode_3d(CUtensorMap* map, const void* base, CUtensorMapDataType type, uint64_t d0,
+               uint64_t d1, uint64_t d2, uint64_t stride1, uint64_t stride2, uint32_t b0,
+               uint32_t b1, uint32_t b2, CUtensorMapSwizzle swizzle,
+               CUtensorMapL2promotion promotion) {
+  auto fn = tensor_map_encoder();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {stride1, stride2};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, type, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, promotion,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -282,7 +301,7 @@ bool plan_gemv(int M, int N, int K, int bits, int group, const DeviceInfo& dev, 
 
 template <int BITS, bool SYM, int G, int MT, int MEFF, bool FAST>
 cudaError_t launch_gemv_t(GemvPlan& plan, const DeviceInfo& dev, const void* codes,
-                          const void* scales, const void* zeros, cudaStream_t s) {
+                          const void* scales, const void* zeros, cudaStream_t s, bool pdl) {
   auto kernel = &wq::gemv::gemv_kernel<BITS, SYM, G, MT, MEFF, FAST>;
   static int configured_smem[kMaxDevices] = {};  // per instantiation and device
   int device = 0;
@@ -298,7 +317,7 @@ cudaError_t launch_gemv_t(GemvPlan& plan, const DeviceInfo& dev, const void* cod
   }
 
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attrs[1];
+  cudaLaunchAttribute attrs[2];
   cfg.blockDim = dim3(wq::gemv::kThreads, 1, 1);
   cfg.stream = s;
   if (plan.C > 1) {
@@ -329,6 +348,12 @@ cudaError_t launch_gemv_t(GemvPlan& plan, const DeviceInfo& dev, const void* cod
   }
   cfg.gridDim = dim3(unsigned(plan.grid), 1, 1);
   cfg.dynamicSmemBytes = plan.smem;
+  if (pdl) {
+    attrs[cfg.numAttrs].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[cfg.numAttrs].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attrs;
+    ++cfg.numAttrs;
+  }
 
   const Params& p = plan.p;
   const int row_bytes = p.K * BITS / 8;
@@ -353,29 +378,203 @@ cudaError_t launch_gemv_t(GemvPlan& plan, const DeviceInfo& dev, const void* cod
 template <int BITS, bool SYM, int G>
 struct GemvOp {
   static cudaError_t run(GemvPlan* plan, const DeviceInfo* dev, const void* c, const void* sc,
-                         const void* z, cudaStream_t s) {
+                         const void* z, cudaStream_t s, bool pdl) {
     // M <= 8: one n8 tile whose columns hold up to 8/MEFF groups of MEFF rows
     const int M = plan->p.M;
     // the unrolled path: one stage per item with the format's natural box count
     const bool fast = M <= 8 && plan->p.stages_per_item == 1 &&
                       plan->p.BPW == wq::gemv::FastShape<BITS>::kBPW;
     if (fast) {
-      if (M == 1) return launch_gemv_t<BITS, SYM, G, 1, 1, true>(*plan, *dev, c, sc, z, s);
-      if (M == 2) return launch_gemv_t<BITS, SYM, G, 1, 2, true>(*plan, *dev, c, sc, z, s);
-      if (M <= 4) return launch_gemv_t<BITS, SYM, G, 1, 4, true>(*plan, *dev, c, sc, z, s);
-      return launch_gemv_t<BITS, SYM, G, 1, 8, true>(*plan, *dev, c, sc, z, s);
+      if (M == 1) return launch_gemv_t<BITS, SYM, G, 1, 1, true>(*plan, *dev, c, sc, z, s, pdl);
+      if (M == 2) return launch_gemv_t<BITS, SYM, G, 1, 2, true>(*plan, *dev, c, sc, z, s, pdl);
+      if (M <= 4) return launch_gemv_t<BITS, SYM, G, 1, 4, true>(*plan, *dev, c, sc, z, s, pdl);
+      return launch_gemv_t<BITS, SYM, G, 1, 8, true>(*plan, *dev, c, sc, z, s, pdl);
     }
-    if (M == 1) return launch_gemv_t<BITS, SYM, G, 1, 1, false>(*plan, *dev, c, sc, z, s);
-    if (M == 2) return launch_gemv_t<BITS, SYM, G, 1, 2, false>(*plan, *dev, c, sc, z, s);
-    if (M <= 4) return launch_gemv_t<BITS, SYM, G, 1, 4, false>(*plan, *dev, c, sc, z, s);
-    if (M <= 8) return launch_gemv_t<BITS, SYM, G, 1, 8, false>(*plan, *dev, c, sc, z, s);
-    if (M <= 16) return launch_gemv_t<BITS, SYM, G, 2, 8, false>(*plan, *dev, c, sc, z, s);
-    return launch_gemv_t<BITS, SYM, G, 4, 8, false>(*plan, *dev, c, sc, z, s);
+    if (M == 1) return launch_gemv_t<BITS, SYM, G, 1, 1, false>(*plan, *dev, c, sc, z, s, pdl);
+    if (M == 2) return launch_gemv_t<BITS, SYM, G, 1, 2, false>(*plan, *dev, c, sc, z, s, pdl);
+    if (M <= 4) return launch_gemv_t<BITS, SYM, G, 1, 4, false>(*plan, *dev, c, sc, z, s, pdl);
+    if (M <= 8) return launch_gemv_t<BITS, SYM, G, 1, 8, false>(*plan, *dev, c, sc, z, s, pdl);
+    if (M <= 16) return launch_gemv_t<BITS, SYM, G, 2, 8, false>(*plan, *dev, c, sc, z, s, pdl);
+    return launch_gemv_t<BITS, SYM, G, 4, 8, false>(*plan, *dev, c, sc, z, s, pdl);
   }
 };
 
+// ------------------------------------------------------- balanced kernel
+
+struct SkPlan {
+  wq::sk::Params p;
+  int grid = 1;
+  size_t smem = 0;
+  int resident = 0;     // B fragments loaded once (all of K in one 16-slice block)
+  int max_stages = 0;   // most stages any CTA walks
+  int max_tiles = 0;    // most row tiles any CTA touches
+};
+
+// Which small-batch kernel wq_matmul uses: 0 chooses, 1 forces the
+// cluster-split kernel, 2 forces the balanced kernel, 3 forces it with split
+// row tiles (tuning and tests).
+int g_kernel_choice = 0;
+
+// Plan the balanced kernel; false if the shape is outside its scope (M <= 8,
+// K a multiple of one 128-byte slice of codes, groups a multiple of 8 per
+// row, activations resident in shared memory next to a ring of >= 3 stages).
+bool plan_sk(int M, int N, int K, int bits, int group, bool symmetric, const DeviceInfo& dev,
+             bool split, SkPlan* plan) {
+  using namespace wq::sk;
+  auto round_up = [](size_t a, size_t b) { return (a + b - 1) / b * b; };
+  if (M < 1 || M > 8) return false;
+  const int slice_k = kSliceBytes * 8 / bits;
+  if (K % slice_k != 0 || group > slice_k) return false;
+  const int ngroups = K / group;
+  if (ngroups % kBlockGroups != 0) return false;
+  const int nk = K / slice_k;
+  const int tiles = (N + kRows - 1) / kRows;
+  const long long units = (long long)tiles * nk;
+  const int gps = slice_k / group;
+  const int meta_blocks = kSlicesPerStage * gps / kBlockGroups;
+
+  wq::sk::Params& p = plan->p;
+  p = wq::sk::Params{};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.ngroups = ngroups;
+  p.tiles = tiles;
+  p.nk = nk;
+  p.split = split ? 1 : 0;
+  p.ctas = int(split ? std::min<long long>(dev.sms, units) : std::min(dev.sms, tiles));
+  p.waves = tiles / p.ctas;
+  p.tail_tiles = tiles % p.ctas;
+
+  // walk every CTA's stages as the kernel does
+  int max_stages = 0, max_tiles = 0;
+  for (int c = 0; c < p.ctas; ++c) {
+    int n = 0, nt = 0;
+    for_each_stage(c, p, [&](const Stage&, bool tile_end) {
+      ++n;
+      nt += tile_end ? 1 : 0;
+    });
+    max_stages = std::max(max_stages, n);
+    max_tiles = std::max(max_tiles, nt);
+  }
+  plan->max_stages = max_stages;
+  plan->max_tiles = max_tiles;
+  plan->resident = nk <= kSlicesPerStage ? 1 : 0;
+  p.box_slices = std::min(kSlicesPerStage, nk);
+  p.box_blocks = std::min(meta_blocks, ngroups / kBlockGroups);
+
+  const size_t meta_bytes = size_t(meta_blocks) * kBlockBytes * (symmetric ? 1 : 2);
+  p.stage_bytes = uint32_t(round_up(kCodesStage + meta_bytes, 1024));
+  // activation rows an odd multiple of 64 bytes apart (bank halves alternate)
+  p.x_stride = uint32_t(2 * K + (((2 * K) / 64) % 2 == 0 ? 64 : 0));
+  const size_t fixed_x = round_up(size_t(M) * p.x_stride, 128);
+  const size_t fixed_sx = round_up(size_t(M) * ngroups * 8, 128);  // {2^-sigma, sum} per group
+  const size_t per_slot = size_t(kWarps) * kRows * M * 4;
+  p.red_mode = size_t(max_tiles) * per_slot <= 32 * 1024 ? 0 : 2;
+  const size_t fixed_red = round_up((p.red_mode == 0 ? max_tiles : 2) * per_slot, 128);
+  const size_t head = 1024;  // barriers and the abort flag
+  const size_t fixed = head + fixed_x + fixed_sx + fixed_red;
+  const size_t budget = size_t(dev.max_smem_optin);
+  if (fixed + p.stage_bytes > budget) return false;
+  int depth = int((budget - fixed) / p.stage_bytes);
+  depth = std::min(depth, std::min(kMaxDepth, max_stages));
+  if (depth < std::min(3, max_stages)) return false;
+  p.depth = depth;
+  p.off_ring = uint32_t(head);
+  p.off_x = uint32_t(head + size_t(depth) * p.stage_bytes);
+  p.off_sx = uint32_t(p.off_x + fixed_x);
+  p.off_red = uint32_t(p.off_sx + fixed_sx);
+  plan->smem = p.off_red + fixed_red;
+  plan->grid = p.ctas;
+  return true;
+}
+
+template <int BITS, bool SYM, int G, int MEFF, bool RES>
+cudaError_t launch_sk_t(SkPlan& plan, const DeviceInfo& dev, const void* codes,
+                        const void* scales, const void* zeros, cudaStream_t s, bool pdl) {
+  using namespace wq::sk;
+  auto kernel = &gemv_sk_kernel<BITS, SYM, G, MEFF, RES>;
+  static int configured[kMaxDevices] = {};
+  int device = 0;
+  cudaGetDevice(&device);
+  if (device < 0 || device >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (configured[device] == 0) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         dev.max_smem_optin);
+    if (e != cudaSuccess) return e;
+    configured[device] = 1;
+  }
+  const wq::sk::Params& p = plan.p;
+  const uint64_t row_bytes = uint64_t(p.K) * BITS / 8;
+  const uint64_t nblk = uint64_t(p.ngroups) / kBlockGroups;
+  CUtensorMap c16, c1, s16, s1, z16, z1;
+  if (!encode_3d(&c16, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, kSliceBytes, uint64_t(p.N),
+                 uint64_t(p.nk), row_bytes, kSliceBytes, kSliceBytes, kRows,
+                 uint32_t(p.box_slices), CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
+      !encode_3d(&c1, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, kSliceBytes, uint64_t(p.N),
+                 uint64_t(p.nk), row_bytes, kSliceBytes, kSliceBytes, kRows, 1,
+                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) ||
+      !encode_3d(&s16, scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, kBlockGroups, uint64_t(p.N), nblk,
+                 uint64_t(p.ngroups) * 2, kBlockGroups * 2, kBlockGroups, kRows,
+                 uint32_t(p.box_blocks), CU_TENSOR_MAP_SWIZZLE_NONE,
+                 CU_TENSOR_MAP_L2_PROMOTION_NONE) ||
+      !encode_3d(&s1, scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, kBlockGroups, uint64_t(p.N), nblk,
+                 uint64_t(p.ngroups) * 2, kBlockGroups * 2, kBlockGroups, kRows, 1,
+                 CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE))
+    return cudaErrorInvalidValue;
+  std::memcpy(&z16, &s16, sizeof(s16));
+  std::memcpy(&z1, &s1, sizeof(s1));
+  if (!SYM &&
+      (!encode_3d(&z16, zeros, CU_TENSOR_MAP_DATA_TYPE_UINT16, kBlockGroups, uint64_t(p.N), nblk,
+                  uint64_t(p.ngroups) * 2, kBlockGroups * 2, kBlockGroups, kRows,
+                  uint32_t(p.box_blocks), CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE) ||
+       !encode_3d(&z1, zeros, CU_TENSOR_MAP_DATA_TYPE_UINT16, kBlockGroups, uint64_t(p.N), nblk,
+                  uint64_t(p.ngroups) * 2, kBlockGroups * 2, kBlockGroups, kRows, 1,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE)))
+    return cudaErrorInvalidValue;
+
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attrs[1];
+  cfg.gridDim = dim3(unsigned(plan.grid), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = plan.smem;
+  cfg.stream = s;
+  plan.p.pdl = pdl ? 1 : 0;
+  if (pdl) {
+    attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attrs;
+    cfg.numAttrs = 1;
+  }
+  return cudaLaunchKernelEx(&cfg, kernel, c16, c1, s16, s1, z16, z1, plan.p);
+}
+
+template <int BITS, bool SYM, int G>
+struct SkOp {
+  static cudaError_t run(SkPlan* plan, const DeviceInfo* dev, const void* c, const void* sc,
+                         const void* z, cudaStream_t s, bool pdl) {
+    const int M = plan->p.M;
+    if (plan->resident) {
+      if (M == 1) return launch_sk_t<BITS, SYM, G, 1, true>(*plan, *dev, c, sc, z, s, pdl);
+      if (M == 2) return launch_sk_t<BITS, SYM, G, 2, true>(*plan, *dev, c, sc, z, s, pdl);
+      if (M <= 4) return launch_sk_t<BITS, SYM, G, 4, true>(*plan, *dev, c, sc, z, s, pdl);
+      return launch_sk_t<BITS, SYM, G, 8, true>(*plan, *dev, c, sc, z, s, pdl);
+    }
+    if (M == 1) return launch_sk_t<BITS, SYM, G, 1, false>(*plan, *dev, c, sc, z, s, pdl);
+    if (M == 2) return launch_sk_t<BITS, SYM, G, 2, false>(*plan, *dev, c, sc, z, s, pdl);
+    if (M <= 4) return launch_sk_t<BITS, SYM, G, 4, false>(*plan, *dev, c, sc, z, s, pdl);
+    return launch_sk_t<BITS, SYM, G, 8, false>(*plan, *dev, c, sc, z, s, pdl);
+  }
+};
+
+// The last CUDA error a call returned (reported by an internal export).
+cudaError_t g_last_cuda_error = cudaSuccess;
+
 wq_status from_cuda(cudaError_t e) {
   if (e == cudaSuccess) return WQ_OK;
+  g_last_cuda_error = e;
   if (e == cudaErrorInvalidValue) return WQ_ERR_INVALID_ARG;
   if (e == cudaErrorNotSupported) return WQ_ERR_UNSUPPORTED;
   return WQ_ERR_CUDA;
@@ -429,21 +628,60 @@ wq_status wq_dequantize(const void* codes, const void* scales, const void* zeros
   return from_cuda(e);
 }
 
+size_t wq_matmul_workspace_bytes(void) {
+  return size_t(wq::sk::kWsCtasMax) * (wq::sk::kWsRowsMax * 4 + 4);
+}
+
 wq_status wq_matmul(const void* X, int64_t M, const void* codes, const void* scales,
                     const void* zeros, int64_t N, int64_t K, int bits, int group, int symmetric,
-                    void* Y, int out_dtype, wq_stream_t stream) {
+                    void* Y, int out_dtype, void* workspace, size_t workspace_bytes,
+                    unsigned int flags, wq_stream_t stream) {
   if (!valid_format(N, K, bits, group) || M < 1 || M >= (int64_t(1) << 31))
     return WQ_ERR_INVALID_ARG;
   if (symmetric != 0 && symmetric != 1) return WQ_ERR_INVALID_ARG;
   if (out_dtype != WQ_OUT_F32 && out_dtype != WQ_OUT_BF16) return WQ_ERR_INVALID_ARG;
+  if ((flags & ~unsigned(WQ_MATMUL_STATIC_WEIGHTS)) != 0) return WQ_ERR_INVALID_ARG;
   if (!X || !codes || !scales || !Y || (symmetric ? zeros != nullptr : zeros == nullptr))
     return WQ_ERR_INVALID_ARG;
+  if (workspace == nullptr && workspace_bytes != 0) return WQ_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(codes) || !aligned16(scales) || !aligned16(Y) ||
-      (zeros && !aligned16(zeros)))
+      (zeros && !aligned16(zeros)) || (workspace && !aligned16(workspace)))
     return WQ_ERR_ALIGNMENT;
   if (M > 32) return WQ_ERR_UNSUPPORTED;
   DeviceInfo dev;
   if (!device_info(&dev)) return WQ_ERR_CUDA;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool have_ws = workspace != nullptr && workspace_bytes >= wq_matmul_workspace_bytes() &&
+                       dev.sms <= wq::sk::kWsCtasMax;
+
+  // Kernel choice (measured on B200): the balanced kernel for 8-bit codes,
+  // group 32, and layers with fewer than three waves of row tiles per SM;
+  // the cluster-split kernel otherwise.  Splitting row tiles across CTAs
+  // through the workspace measured slower than whole tiles on every shape
+  // tried (the end-of-kernel gather costs more than the balance gains), so
+  // it is used only when forced through the tuning hook.
+  const bool pdl = (flags & WQ_MATMUL_STATIC_WEIGHTS) != 0;
+  const int tiles = int((N + 15) / 16);
+  const bool prefer_balanced = bits == 8 || group == 32 || tiles < 3 * dev.sms;
+  const bool use_balanced =
+      g_kernel_choice >= 2 || (g_kernel_choice == 0 && prefer_balanced);
+  const bool split = have_ws && g_kernel_choice == 3;
+  SkPlan sk;
+  if (use_balanced &&
+      plan_sk(int(M), int(N), int(K), bits, group, symmetric != 0, dev, split, &sk)) {
+    sk.p.X = static_cast<const __nv_bfloat16*>(X);
+    sk.p.Y = Y;
+    sk.p.y_bf16 = out_dtype == WQ_OUT_BF16;
+    if (split) {
+      sk.p.ws_flag = static_cast<unsigned int*>(workspace);
+      sk.p.ws_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                              size_t(wq::sk::kWsCtasMax) * 4);
+    }
+    return from_cuda(dispatch_format<SkOp>(bits, symmetric != 0, group, &sk, &dev, codes, scales,
+                                           zeros, s, pdl));
+  }
+  if (g_kernel_choice >= 2) return WQ_ERR_UNSUPPORTED;
+
   GemvPlan plan;
   if (!plan_gemv(int(M), int(N), int(K), bits, group, dev, 0, &plan)) return WQ_ERR_UNSUPPORTED;
   plan.p.X = static_cast<const __nv_bfloat16*>(X);
@@ -453,8 +691,7 @@ wq_status wq_matmul(const void* X, int64_t M, const void* codes, const void* sca
   plan.p.codes = static_cast<const uint8_t*>(codes);
   plan.p.y_bf16 = out_dtype == WQ_OUT_BF16;
   const cudaError_t e = dispatch_format<GemvOp>(bits, symmetric != 0, group, &plan, &dev, codes,
-                                                scales, zeros,
-                                                reinterpret_cast<cudaStream_t>(stream));
+                                                scales, zeros, s, pdl);
   return from_cuda(e);
 }
 
@@ -487,6 +724,39 @@ void wq_internal_force_gemv_plan(int C, int bpw, int depth) {
   g_force_C = C;
   g_force_bpw = bpw;
   g_force_depth = depth;
+}
+
+// Diagnostic hook, not part of the public ABI: the name of the last CUDA
+// error behind a WQ_ERR_CUDA status.
+const char* wq_internal_last_cuda_error(void) { return cudaGetErrorName(g_last_cuda_error); }
+
+// Tuning and test hook, not part of the public ABI: 0 lets wq_matmul choose
+// the small-batch kernel, 1 forces the cluster-split kernel, 2 forces the
+// balanced kernel, 3 forces the balanced kernel with row tiles split across
+// CTAs whenever a workspace is given (2 and 3 return WQ_ERR_UNSUPPORTED
+// where the balanced kernel does not apply).
+void wq_internal_set_kernel(int choice) { g_kernel_choice = choice; }
+
+// Test hook, not part of the public ABI: the balanced kernel's plan for a
+// device with `sms` SMs and `smem_optin` bytes of shared memory per block,
+// written to out[0..24] (see tests/test_plan_sk.py for the field order).
+// Returns 0 if the shape is outside the kernel's scope.
+int wq_internal_plan_sk(int M, int N, int K, int bits, int group, int symmetric, int sms,
+                        int smem_optin, int split, int64_t* out) {
+  DeviceInfo dev;
+  dev.sms = sms;
+  dev.max_smem_optin = smem_optin;
+  SkPlan plan;
+  if (!plan_sk(M, N, K, bits, group, symmetric != 0, dev, split != 0, &plan)) return 0;
+  const wq::sk::Params& p = plan.p;
+  const int64_t v[] = {p.M,           p.N,          p.K,           p.ngroups,   p.tiles,
+                       p.nk,          p.waves,      p.ctas,        p.split,     p.depth,
+                       p.red_mode,    p.stage_bytes, p.off_ring,   p.off_x,     p.off_sx,
+                       p.off_red,     p.x_stride,   p.box_slices,  p.box_blocks, int64_t(plan.smem),
+                       plan.grid,     plan.resident, plan.max_stages, plan.max_tiles,
+                       p.tail_tiles};
+  for (size_t i = 0; i < sizeof(v) / sizeof(v[0]); ++i) out[i] = v[i];
+  return 1;
 }
 
 // Test hook, not part of the public ABI: the matmul plan for a device with
