@@ -148,6 +148,26 @@ wq_status wq_matmul(const void *X, int64_t M, const void *codes, const void *sca
                     int symmetric, void *Y, int out_dtype, void *workspace,
                     size_t workspace_bytes, unsigned int flags, wq_stream_t stream);
 
+/* As wq_matmul, without a workspace argument and without allocating: the
+ * workspace is a fixed block of device memory inside the library
+ * (wq_matmul_noalloc_scratch_bytes() bytes, zero at load, left zero by every
+ * completed call), found with cudaGetSymbolAddress on the first call on
+ * each device and cleared then.  The pages have no counterpart of this entry
+ * point; it exists for callers that must not allocate (for example inside a
+ * captured CUDA graph).
+ *   - Make the first call on a device before any stream capture (the look-up
+ *     and the clearing are synchronous).
+ *   - All calls on a device share the block: calls whose kernels overlap on
+ *     the GPU (different streams, or graphs replayed concurrently) race.
+ *   - A device with more SMs than the block has room for gets
+ *     WQ_ERR_UNSUPPORTED, as does a workspace larger than the block.
+ * Results are bit-identical to wq_matmul given a workspace. */
+size_t wq_matmul_noalloc_scratch_bytes(void);
+wq_status wq_matmul_noalloc(const void *X, int64_t M, const void *codes, const void *scales,
+                            const void *zeros, int64_t N, int64_t K, int bits, int group,
+                            int symmetric, void *Y, int out_dtype, unsigned int flags,
+                            wq_stream_t stream);
+
 /* Read and clear the device status word (WQ_OK if no kernel recorded an
  * error).  Synchronizes `stream` first. */
 wq_status wq_get_device_error(wq_stream_t stream);

@@ -61,6 +61,11 @@ def _load() -> ctypes.CDLL:
     lib.wq_matmul.argtypes = [vp, i64, vp, vp, vp, i64, i64, i32, i32, i32, vp, i32, vp, sz,
                               ctypes.c_uint, vp]
     lib.wq_matmul.restype = i32
+    lib.wq_matmul_noalloc.argtypes = [vp, i64, vp, vp, vp, i64, i64, i32, i32, i32, vp, i32,
+                                      ctypes.c_uint, vp]
+    lib.wq_matmul_noalloc.restype = i32
+    lib.wq_matmul_noalloc_scratch_bytes.argtypes = []
+    lib.wq_matmul_noalloc_scratch_bytes.restype = sz
     lib.wq_get_device_error.argtypes = [vp]
     lib.wq_get_device_error.restype = i32
     lib.wq_status_string.argtypes = [i32]
@@ -219,6 +224,25 @@ def matmul(X: torch.Tensor, qw: QuantizedWeight, out_dtype: torch.dtype = torch.
         out.copy_(Yd, non_blocking=True)
         return out
     return Yd.cpu()
+
+
+def matmul_noalloc(X: torch.Tensor, qw: QuantizedWeight, out_dtype: torch.dtype = torch.float32,
+                   out: torch.Tensor | None = None, static_weights: bool = False) -> torch.Tensor:
+    """``wq_matmul_noalloc``: as ``matmul`` with device tensors, the workspace
+    being the library's own fixed block (see ``include/wq.h``)."""
+    if X.dtype != torch.bfloat16 or X.dim() != 2 or X.shape[1] != qw.K:
+        raise ValueError("X must be a 2-D bfloat16 tensor [M, K]")
+    _require_cuda(X, qw.codes, qw.scales, qw.zeros)
+    dev = qw.codes.device
+    M = X.shape[0]
+    Y = out if out is not None else torch.empty((M, qw.N), dtype=out_dtype, device=dev)
+    _require_cuda(Y)
+    _check(lib.wq_matmul_noalloc(_ptr(X), M, _ptr(qw.codes), _ptr(qw.scales), _ptr(qw.zeros),
+                                 qw.N, qw.K, qw.bits, qw.group, int(qw.symmetric), _ptr(Y),
+                                 WQ_OUT_BF16 if Y.dtype == torch.bfloat16 else WQ_OUT_F32,
+                                 WQ_MATMUL_STATIC_WEIGHTS if static_weights else 0,
+                                 _stream(dev)), "wq_matmul_noalloc")
+    return Y
 
 
 def get_device_error(device: torch.device | None = None) -> int:

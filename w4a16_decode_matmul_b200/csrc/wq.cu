@@ -695,6 +695,59 @@ wq_status wq_matmul(const void* X, int64_t M, const void* codes, const void* sca
   return from_cuda(e);
 }
 
+// ------------------------------------------------------ no-allocation entry
+
+}  // extern "C"
+
+namespace {
+
+// Scratch of wq_matmul_noalloc: the matmul workspace of any call (flags for
+// kWsCtasMax CTAs and their binary32 partial sums, M <= 8), in device memory
+// that the module brings with it.  Zero at load; every completed call leaves
+// it zero.
+constexpr size_t kNoallocScratchBytes =
+    size_t(wq::sk::kWsCtasMax) * (size_t(wq::sk::kWsRowsMax) * 4 + 4);
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+void* g_noalloc_address[kMaxDevices] = {};
+
+// The scratch address on the current device, looked up once per device (with
+// that device current) and cleared once; null on failure.
+void* noalloc_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (g_noalloc_address[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return nullptr;
+    if (cudaMemset(p, 0, kNoallocScratchBytes) != cudaSuccess) return nullptr;
+    g_noalloc_address[dev] = p;
+  }
+  return g_noalloc_address[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t wq_matmul_noalloc_scratch_bytes(void) { return kNoallocScratchBytes; }
+
+wq_status wq_matmul_noalloc(const void* X, int64_t M, const void* codes, const void* scales,
+                            const void* zeros, int64_t N, int64_t K, int bits, int group,
+                            int symmetric, void* Y, int out_dtype, unsigned int flags,
+                            wq_stream_t stream) {
+  // the scratch holds any workspace the matmul asks for; refuse otherwise
+  if (wq_matmul_workspace_bytes() > kNoallocScratchBytes) return WQ_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  if (!device_info(&dev)) return WQ_ERR_CUDA;
+  if (dev.sms > wq::sk::kWsCtasMax) return WQ_ERR_UNSUPPORTED;
+  void* scratch = noalloc_scratch();
+  if (scratch == nullptr) return WQ_ERR_CUDA;
+  return wq_matmul(X, M, codes, scales, zeros, N, K, bits, group, symmetric, Y, out_dtype,
+                   scratch, kNoallocScratchBytes, flags, stream);
+}
+
 wq_status wq_get_device_error(wq_stream_t stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return WQ_ERR_CUDA;
