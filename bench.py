@@ -298,6 +298,10 @@ def run_wq(args):
     # end to end through the public API: host X in, host Y out, every step
     e2e = measure_e2e(wq, torch, dev, pool, pool_n, args)
 
+    # the prefill row (tensor cores), outside the timed region
+    del pool
+    prefill = prefill_points(wq, torch, dev)
+
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
         "steps": steps, "warmup": max(args.warmup, 3), "ms_per_step": ms / steps,
@@ -320,6 +324,7 @@ def run_wq(args):
         "e2e": e2e,
         "device_status": err,
         **extra,
+        "prefill_tcgen05": prefill,
     }
     if world == 1:
         gbs, st, el = time_oracle(10.0)
@@ -373,6 +378,51 @@ def compare_points(wq, torch, dev, stream, pool, X, pool_n, reps: int = 50):
     }
 
 
+def prefill_points(wq, torch, dev, reps: int = 8):
+    """The prefill-shaped matmul (M in {512, 2048, 8192}, K=4096, N=14336,
+    INT4 asymmetric group 128) on the tensor cores next to a dense bf16 GEMM
+    of the same shape (torch/cuBLAS); TFLOP/s = 2 M N K / time, and the
+    fraction of the measured dense bf16 peak (burst)."""
+    import synth
+    qw = wq.quantize(synth.weight(N, K, seed=0).to(dev), bits=BITS, group=GROUP, symmetric=SYM)
+    Wd = torch.randn(N, K, device=dev, dtype=torch.bfloat16)
+    peak = measured_bf16_tflops()
+    out = {}
+    for m in (512, 2048, 8192):
+        X = synth.activation(m, K, seed=3).to(dev)
+        Y = torch.empty(m, N, device=dev, dtype=torch.float32)
+        Yd = torch.empty(m, N, device=dev, dtype=torch.bfloat16)
+
+        def timed(fn):
+            for _ in range(2):
+                fn()
+            torch.cuda.synchronize(dev)
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            for _ in range(reps):
+                fn()
+            e.record()
+            torch.cuda.synchronize(dev)
+            return s.elapsed_time(e) / reps * 1e3
+
+        us = timed(lambda: wq.matmul(X, qw, out=Y))
+        dus = timed(lambda: torch.matmul(X, Wd.T, out=Yd))
+        fl = 2.0 * m * N * K
+        out[str(m)] = {"us": round(us, 1), "tflops": round(fl / us / 1e6, 1),
+                       "frac_of_measured_bf16": round(fl / us / 1e6 / peak, 4),
+                       "dense_bf16_us": round(dus, 1), "dense_bf16_tflops": round(fl / dus / 1e6, 1)}
+        del X, Y, Yd
+    return out
+
+
+def measured_bf16_tflops():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"])
+    return 1590.0
+
+
 def measure_e2e(wq, torch, dev, pool, pool_n, args):
     """Public API with host buffers: pinned X copied in, Y read back, every
     step, inside the timed region."""
@@ -403,7 +453,8 @@ def measure_e2e(wq, torch, dev, pool, pool_n, args):
 
 def ncu_case():
     """A small, self-contained launch sequence for ncu captures: one
-    quantize of the benchmark layer, then 8 fused matmuls on it."""
+    quantize of the benchmark layer, 8 fused decode matmuls (M=1) on it,
+    then 2 prefill matmuls (M=2048) on it."""
     import torch
     import synth
     import w4a16_decode_matmul_b200 as wq
@@ -413,6 +464,10 @@ def ncu_case():
     Y = torch.empty(M, N, dtype=torch.float32, device=dev)
     for _ in range(8):
         wq.matmul(X, qw, out=Y)
+    Xp = synth.activation(2048, K, seed=2).to(dev)
+    Yp = torch.empty(2048, N, dtype=torch.float32, device=dev)
+    for _ in range(2):
+        wq.matmul(Xp, qw, out=Yp)
     torch.cuda.synchronize(dev)
     assert wq.get_device_error(dev) == 0
     print("ncu case ok")
@@ -426,7 +481,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=2000)
     ap.add_argument("--impl", choices=["wq", "reference"], default="wq")
     ap.add_argument("--ncu-case", action="store_true",
-                    help="no timing: quantize the layer and run 8 fused matmuls, for ncu")
+                    help="no timing: quantize the layer, run 8 decode and 2 prefill matmuls, for ncu")
     args = ap.parse_args(argv)
     if args.ncu_case:
         return ncu_case()
