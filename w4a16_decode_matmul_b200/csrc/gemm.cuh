@@ -12,19 +12,22 @@
 // D_g = sum over the group of x (q - z) is scaled in binary32:
 // y = sum_g s_g D_g.  Products are exact; D_g accumulates in binary32.
 //
-// One CTA computes a 128 x 128 tile of Y over all of K, per stage of 64 k:
+// One CTA computes a 128 x 128 tile of Y over all of K, per stage of 64 k
+// (a ring of 4 stages, each holding the activation tile, the codes and the
+// dequantized weight tile):
 //   warp 0      TMA: the 128 x 64 activation tile (128-byte swizzle) and the
 //               128 rows x 64 codes; once per tile the tile's scales/zeros;
-//   warps 2-5   dequantize: one row of codes per thread -> 64 bfloat16
+//   warps 2-9   dequantize: half a row of codes per thread -> 32 bfloat16
 //               (q - z) written in the same swizzled K-major layout, then an
 //               async-proxy fence and an arrive;
 //   warp 1      one thread issues tcgen05.mma (M=128, N=128, K=16, bfloat16
 //               in, binary32 accumulator in tensor memory) per 16 k; a
-//               group's MMAs accumulate into one of two 128-column TMEM
+//               group's MMAs accumulate into one of three 128-column TMEM
 //               buffers, whose commit hands it to the epilogue;
-//   warps 6-13  epilogue: each thread owns one row and 64 columns; per group
+//   warps 10-17 epilogue: each thread owns one row and 64 columns; per group
 //               it reads D_g from TMEM, releases the buffer and adds s_g D_g
-//               into registers (binary32); at the end it writes Y.
+//               into the running sum S, kept in TMEM next to the group
+//               buffers (binary32); at the end it writes S to Y.
 // Every wait is bounded in time; a timeout records WQ_ERR_TIMEOUT, the other
 // roles skip their work, issued copies and MMAs are drained and TMEM is freed.
 #pragma once
@@ -38,21 +41,23 @@ constexpr int kBM = 128;                 // rows of X per tile (MMA M)
 constexpr int kBN = 128;                 // rows of W per tile (MMA N)
 constexpr int kBK = 64;                  // k per stage (one 128-byte swizzled row)
 constexpr int kStages = 4;
-constexpr int kDequantWarp0 = 2, kNumDequantWarps = 4;
-constexpr int kEpilogueWarp0 = 6, kNumEpilogueWarps = 8;
-constexpr int kThreads = (kEpilogueWarp0 + kNumEpilogueWarps) * 32;  // 448
+constexpr int kDequantWarp0 = 2, kNumDequantWarps = 8;
+constexpr int kEpilogueWarp0 = 10, kNumEpilogueWarps = 8;
+constexpr int kThreads = (kEpilogueWarp0 + kNumEpilogueWarps) * 32;  // 576
 constexpr int kTileBytes = kBM * kBK * 2;                              // 16 KB (A and B alike)
-constexpr int kTmemCols = 2 * kBN;                                     // two group buffers
+constexpr int kAccBufs = 3;                   // group accumulators in TMEM
+constexpr int kTmemCols = (kAccBufs + 1) * kBN;  // 512: the buffers and the running sum
+constexpr int kSumCol = kAccBufs * kBN;        // first TMEM column of the running sum S
 constexpr int kColsPerThread = kBN / 2;                                // epilogue: 64 columns
 
 // mbarrier slots in the first KB of shared memory
 constexpr int kBarLdFull = 0;            // [kStages] activation + codes tile landed
 constexpr int kBarEmpty = 4;             // [kStages] MMAs of the stage done (commit)
 constexpr int kBarBFull = 8;             // [kStages] dequantized tile written
-constexpr int kBarAccFull = 12;          // [2] group accumulator ready (commit)
-constexpr int kBarAccEmpty = 14;         // [2] group accumulator read
-constexpr int kBarMeta = 16;             // tile's scales / zeros landed
-constexpr int kBarMmaDone = 17;          // every MMA of the CTA finished
+constexpr int kBarAccFull = 12;          // [kAccBufs] group accumulator ready (commit)
+constexpr int kBarAccEmpty = 15;         // [kAccBufs] group accumulator read
+constexpr int kBarMeta = 18;             // tile's scales / zeros landed
+constexpr int kBarMmaDone = 19;          // every MMA of the CTA finished
 constexpr int kTmemSlot = 576;           // byte offset of the TMEM base address
 constexpr int kAbortSlot = 580;          // byte offset of the abort flag
 
@@ -130,6 +135,29 @@ __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31, %32};"
+      ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])),
+      "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])),
+      "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
+      "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
+      "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])),
+      "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
+      "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])),
+      "r"(__float_as_uint(v[23])), "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])),
+      "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])),
+      "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
   uint32_t r;
   asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
@@ -196,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars[kBarEmpty + s], 1);
       mbar_init(&bars[kBarBFull + s], kNumDequantWarps);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kAccBufs; ++b) {
       mbar_init(&bars[kBarAccFull + b], 1);
       mbar_init(&bars[kBarAccEmpty + b], kNumEpilogueWarps);
     }
@@ -262,8 +290,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t b0 = smem_addr(smem + p.off_b);
       int kb = 0;
       for (int gi = 0; gi < p.ngroups && !*abort_flag; ++gi) {
-        const int buf = gi & 1;
-        if (!wait(kBarAccEmpty + buf, (uint32_t(gi >> 1) & 1u) ^ 1u)) break;
+        const int buf = gi % kAccBufs;
+        if (!wait(kBarAccEmpty + buf, (uint32_t(gi / kAccBufs) & 1u) ^ 1u)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + uint32_t(buf * kBN);
         bool ok = true;
@@ -291,7 +319,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < kEpilogueWarp0) {
     // ------------------------------------------------------------ dequantize
-    const int r = threadIdx.x - kDequantWarp0 * 32;  // row of the W tile, 0..127
+    const int dt = threadIdx.x - kDequantWarp0 * 32;  // 0..255
+    const int r = dt & (kBN - 1);                     // row of the W tile
+    const int part = dt >> 7;                         // 16-byte chunks 4*part .. 4*part+3
     const bool have_meta = wait(kBarMeta, 0);
     const __half* zrow = reinterpret_cast<const __half*>(smem + p.off_meta_z) + r * p.ngroups;
     for (int kb = 0; kb < nkb && have_meta; ++kb) {
@@ -306,23 +336,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (BITS == 4) {
         const __nv_bfloat162 zz = __floats2bfloat162_rn(128.f + zc, 128.f + zc);
         const uint32_t zc2 = *reinterpret_cast<const uint32_t*>(&zz);
-        const uint4 c0 = *reinterpret_cast<const uint4*>(crow);
-        const uint4 c1 = *reinterpret_cast<const uint4*>(crow + 16);
-        const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        const uint4 c = *reinterpret_cast<const uint4*>(crow + 16 * part);
+        const uint32_t w[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {  // word j: k = 8j .. 8j + 7 = 16-byte chunk j
+        for (int j = 0; j < 4; ++j) {  // word j: k = 8j .. 8j + 7 of this half = chunk 4*part + j
           uint32_t o[4];
           dequant_u4_kord(w[j], zc2, o);
-          *reinterpret_cast<uint4*>(brow + ((j ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+          const int ch = 4 * part + j;
+          *reinterpret_cast<uint4*>(brow + ((ch ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
         }
       } else {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {  // 8 bytes of codes -> 16-byte chunk j
-          const uint2 c = *reinterpret_cast<const uint2*>(crow + 8 * j);
+        for (int j = 0; j < 4; ++j) {  // 8 bytes of codes -> 16-byte chunk 4*part + j
+          const int ch = 4 * part + j;
+          const uint2 c = *reinterpret_cast<const uint2*>(crow + 8 * ch);
           uint32_t o0[2], o1[2];
           dequant_u8_kord(c.x, zc, o0);
           dequant_u8_kord(c.y, zc, o1);
-          *reinterpret_cast<uint4*>(brow + ((j ^ (r & 7)) << 4)) = make_uint4(o0[0], o0[1], o1[0], o1[1]);
+          *reinterpret_cast<uint4*>(brow + ((ch ^ (r & 7)) << 4)) = make_uint4(o0[0], o0[1], o1[0], o1[1]);
         }
       }
       fence_async_shared();  // the tensor cores read B through the async proxy
@@ -346,68 +377,82 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     named_barrier_sync(2, kNumEpilogueWarps * 32);
-    float acc[kColsPerThread];
-#pragma unroll
-    for (int j = 0; j < kColsPerThread; ++j) acc[j] = 0.f;
+    const uint32_t lanes = uint32_t(32 * quarter) << 16;
+    const uint32_t sum_addr = tmem_base + lanes + uint32_t(kSumCol + half * kColsPerThread);
+    int done = 0;
     for (int gi = 0; gi < p.ngroups && have_meta; ++gi) {
-      const int buf = gi & 1;
-      if (!wait(kBarAccFull + buf, uint32_t(gi >> 1) & 1u)) break;
+      const int buf = gi % kAccBufs;
+      if (!wait(kBarAccFull + buf, uint32_t(gi / kAccBufs) & 1u)) break;
       tc_fence_after();
-      const uint32_t taddr =
-          tmem_base + (uint32_t(32 * quarter) << 16) + uint32_t(buf * kBN + half * kColsPerThread);
-      float d0[32], d1[32];
-      tmem_ld32(taddr, d0);
-      tmem_ld32(taddr + 32, d1);
-      tmem_wait_ld();
+      const uint32_t taddr = tmem_base + lanes + uint32_t(buf * kBN + half * kColsPerThread);
+      const float* sg = stab + gi * kBN + half * kColsPerThread;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {  // 32 columns at a time: S += s_g D_g
+        float d[32], acc[32];
+        tmem_ld32(taddr + 32 * h, d);
+        if (gi > 0) tmem_ld32(sum_addr + 32 * h, acc);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+          const float4 sv = *reinterpret_cast<const float4*>(sg + 32 * h + j);
+          acc[j + 0] = fmaf(sv.x, d[j + 0], gi > 0 ? acc[j + 0] : 0.f);
+          acc[j + 1] = fmaf(sv.y, d[j + 1], gi > 0 ? acc[j + 1] : 0.f);
+          acc[j + 2] = fmaf(sv.z, d[j + 2], gi > 0 ? acc[j + 2] : 0.f);
+          acc[j + 3] = fmaf(sv.w, d[j + 3], gi > 0 ? acc[j + 3] : 0.f);
+        }
+        tmem_st32(sum_addr + 32 * h, acc);
+      }
+      tmem_wait_st();
+      // D_g is read: the MMA warp may overwrite this buffer
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[kBarAccEmpty + buf]);
-      const float* sg = stab + gi * kBN + half * kColsPerThread;
-#pragma unroll
-      for (int j = 0; j < 32; j += 4) {
-        const float4 s0 = *reinterpret_cast<const float4*>(sg + j);
-        const float4 s1 = *reinterpret_cast<const float4*>(sg + 32 + j);
-        acc[j + 0] = fmaf(s0.x, d0[j + 0], acc[j + 0]);
-        acc[j + 1] = fmaf(s0.y, d0[j + 1], acc[j + 1]);
-        acc[j + 2] = fmaf(s0.z, d0[j + 2], acc[j + 2]);
-        acc[j + 3] = fmaf(s0.w, d0[j + 3], acc[j + 3]);
-        acc[32 + j + 0] = fmaf(s1.x, d1[j + 0], acc[32 + j + 0]);
-        acc[32 + j + 1] = fmaf(s1.y, d1[j + 1], acc[32 + j + 1]);
-        acc[32 + j + 2] = fmaf(s1.z, d1[j + 2], acc[32 + j + 2]);
-        acc[32 + j + 3] = fmaf(s1.w, d1[j + 3], acc[32 + j + 3]);
-      }
+      done = gi + 1;
     }
     const int m = m0 + row;
     const int nb = n0 + half * kColsPerThread;
-    if (!*abort_flag && m < p.M) {
-      if (p.Y_f32 != nullptr) {
-        float* yrow = p.Y_f32 + size_t(m) * p.N + nb;
-        if (nb + kColsPerThread <= p.N && (p.N % 4) == 0) {
+    if (!*abort_flag && done == p.ngroups) {
 #pragma unroll
-          for (int j = 0; j < kColsPerThread; j += 4)
-            *reinterpret_cast<float4*>(yrow + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
-        } else {
-          for (int j = 0; j < kColsPerThread && nb + j < p.N; ++j) yrow[j] = acc[j];
-        }
-      } else {
-        __nv_bfloat16* yrow = p.Y_bf16 + size_t(m) * p.N + nb;
-        if (nb + kColsPerThread <= p.N && (p.N % 8) == 0) {
+      for (int h = 0; h < 2; ++h) {
+        float acc[32];
+        tmem_ld32(sum_addr + 32 * h, acc);
+        tmem_wait_ld();
+        const int nh = nb + 32 * h;
+        if (m < p.M) {
+          if (p.Y_f32 != nullptr) {
+            float* yrow = p.Y_f32 + size_t(m) * p.N + nh;
+            if (nh + 32 <= p.N && (p.N % 4) == 0) {
 #pragma unroll
-          for (int j = 0; j < kColsPerThread; j += 8) {
-            uint4 o;
-            __nv_bfloat162 h0 = __floats2bfloat162_rn(acc[j], acc[j + 1]);
-            __nv_bfloat162 h1 = __floats2bfloat162_rn(acc[j + 2], acc[j + 3]);
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[j + 4], acc[j + 5]);
-            __nv_bfloat162 h3 = __floats2bfloat162_rn(acc[j + 6], acc[j + 7]);
-            o.x = *reinterpret_cast<uint32_t*>(&h0);
-            o.y = *reinterpret_cast<uint32_t*>(&h1);
-            o.z = *reinterpret_cast<uint32_t*>(&h2);
-            o.w = *reinterpret_cast<uint32_t*>(&h3);
-            *reinterpret_cast<uint4*>(yrow + j) = o;
+              for (int j = 0; j < 32; j += 4)
+                *reinterpret_cast<float4*>(yrow + j) =
+                    make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (nh + j < p.N) yrow[j] = acc[j];
+            }
+          } else {
+            __nv_bfloat16* yrow = p.Y_bf16 + size_t(m) * p.N + nh;
+            if (nh + 32 <= p.N && (p.N % 8) == 0) {
+#pragma unroll
+              for (int j = 0; j < 32; j += 8) {
+                uint4 o;
+                __nv_bfloat162 h0 = __floats2bfloat162_rn(acc[j], acc[j + 1]);
+                __nv_bfloat162 h1 = __floats2bfloat162_rn(acc[j + 2], acc[j + 3]);
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[j + 4], acc[j + 5]);
+                __nv_bfloat162 h3 = __floats2bfloat162_rn(acc[j + 6], acc[j + 7]);
+                o.x = *reinterpret_cast<uint32_t*>(&h0);
+                o.y = *reinterpret_cast<uint32_t*>(&h1);
+                o.z = *reinterpret_cast<uint32_t*>(&h2);
+                o.w = *reinterpret_cast<uint32_t*>(&h3);
+                *reinterpret_cast<uint4*>(yrow + j) = o;
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (nh + j < p.N) yrow[j] = __float2bfloat16_rn(acc[j]);
+            }
           }
-        } else {
-          for (int j = 0; j < kColsPerThread && nb + j < p.N; ++j)
-            yrow[j] = __float2bfloat16_rn(acc[j]);
         }
       }
     }

@@ -918,7 +918,7 @@ int wq_internal_plan_sk(int M, int N, int K, int bits, int group, int symmetric,
 }
 
 // Test hook, not part of the public ABI: the prefill plan, written to
-// out[0..12] (see tests/test_plan_gemm.py for the field order).  Returns 0
+// out[0..14] (see tests/test_plan_gemm.py for the field order).  Returns 0
 // if the shape is outside the prefill kernel's scope.
 int wq_internal_plan_gemm(int M, int N, int K, int bits, int group, int symmetric,
                           int smem_optin, int64_t* out) {
