@@ -43,7 +43,7 @@ WORKLOAD = ("decode GEMV, Llama-8B gate/up layer: M=1, K=4096, N=14336, INT4 asy
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "gemv_w4a16_m1_k4096_n14336.json")
 KERNEL_SOURCES = [os.path.join(ROOT, "w4a16_decode_matmul_b200", "csrc", f)
-                  for f in ("gemv.cuh", "common.cuh", "wq.cu")]
+                  for f in ("gemv_ld.cuh", "unpack.cuh", "common.cuh", "wq.cu")]
 
 
 def algorithmic_bytes(m: int = M, n: int = N, k: int = K, bits: int = BITS,
@@ -294,13 +294,22 @@ def run_wq(args):
 
     # comparison points on the same GPU (not part of the timed region)
     extra = compare_points(wq, torch, dev, stream, pool, X, pool_n)
+    extra["per_graph_distribution"] = graph_distribution(torch, dev, stream, g_full, pool_n)
+    extra["warm_l2"] = warm_l2_point(wq, torch, dev, stream, pool[0], X)
+    extra["stream_read_ceiling"] = stream_ceiling(wq, torch, dev, stream, pool, pool_n)
+    extra["stream_read_ceiling"]["fused_frac_of_ceiling"] = round(
+        extra["stream_read_ceiling"]["us_per_layer"] / (per_launch_ms * 1e3), 4)
 
     # end to end through the public API: host X in, host Y out, every step
     e2e = measure_e2e(wq, torch, dev, pool, pool_n, args)
 
     # the prefill row (tensor cores), outside the timed region
-    del pool
+    del pool, g_full, g_rest
+    g_full = g_rest = None
     prefill = prefill_points(wq, torch, dev)
+    # the quantize rows: the benchmark layer, then every matrix of the model
+    quant = quantize_points(wq, torch, dev, stream)
+    model_quant = whole_model_quantize(wq, torch, dev, stream)
 
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
@@ -325,6 +334,8 @@ def run_wq(args):
         "device_status": err,
         **extra,
         "prefill_tcgen05": prefill,
+        "quantize_layer": quant,
+        "quantize_whole_model": model_quant,
     }
     if world == 1:
         gbs, st, el = time_oracle(10.0)
@@ -376,6 +387,165 @@ def compare_points(wq, torch, dev, stream, pool, X, pool_n, reps: int = 50):
         "fused_eager_us_per_layer": round(fused_us, 3),
         "fused_vs_dense_speedup": round(dense_us / fused_us, 3),
     }
+
+
+def graph_distribution(torch, dev, stream, graph, pool_n: int, reps: int = 60):
+    """Microseconds per layer of single replays of the timed graph (pool_n
+    launches each): p10 / median / p90 over `reps` replays."""
+    times = []
+    with torch.cuda.stream(stream):
+        for _ in range(reps):
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record(stream)
+            graph.replay()
+            e.record(stream)
+            times.append((s, e))
+    torch.cuda.synchronize(dev)
+    us = sorted(s.elapsed_time(e) * 1e3 / pool_n for s, e in times)
+    pick = lambda q: round(us[min(len(us) - 1, int(q * len(us)))], 3)
+    return {"p10_us": pick(0.1), "median_us": pick(0.5), "p90_us": pick(0.9),
+            "replays": reps, "launches_per_replay": pool_n}
+
+
+def warm_l2_point(wq, torch, dev, stream, qw, X, count: int = 20, reps: int = 20):
+    """The same graph-launched matmul on ONE weight copy (31 MB, resident in
+    the L2 after the first launch): labelled warm-L2, not an HBM figure."""
+    Y = torch.empty(M, N, dtype=torch.float32, device=dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        wq.matmul(X, qw, out=Y, static_weights=True)
+        stream.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(count):
+                wq.matmul(X, qw, out=Y, static_weights=True)
+        g.replay()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e.record(stream)
+    torch.cuda.synchronize(dev)
+    us = s.elapsed_time(e) * 1e3 / (count * reps)
+    return {"us_per_layer": round(us, 3), "gbs": round(algorithmic_bytes() / us / 1e3, 1),
+            "how": "one weight copy, L2-resident: not an HBM number"}
+
+
+def stream_ceiling(wq, torch, dev, stream, pool, pool_n, reps: int = 20):
+    """The practical ceiling at this size: a read-only streaming kernel of
+    the library over the same bytes (codes, scales, zeros of each pool copy),
+    launched back to back from a CUDA graph with programmatic dependent
+    launch, exactly like the timed matmul."""
+    import ctypes
+    lib = wq.lib
+    vp, sz = ctypes.c_void_p, ctypes.c_size_t
+    lib.wq_internal_stream_read.argtypes = [vp, sz, vp, sz, vp, sz, vp, ctypes.c_int, vp]
+    lib.wq_internal_stream_read.restype = ctypes.c_int
+    lib.wq_internal_stream_read_out_bytes.argtypes = []
+    lib.wq_internal_stream_read_out_bytes.restype = sz
+    out = torch.empty(lib.wq_internal_stream_read_out_bytes() // 4, dtype=torch.int32, device=dev)
+
+    def nbytes(t):
+        return 0 if t is None else t.numel() * t.element_size()
+
+    def launch(i):
+        q = pool[i % pool_n]
+        st = lib.wq_internal_stream_read(
+            q.codes.data_ptr(), nbytes(q.codes), q.scales.data_ptr(), nbytes(q.scales),
+            None if q.zeros is None else q.zeros.data_ptr(), nbytes(q.zeros),
+            out.data_ptr(), 1, stream.cuda_stream)
+        if st != 0:
+            raise RuntimeError(f"wq_internal_stream_read: status {st}")
+
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        launch(0)
+        stream.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(pool_n):
+                launch(i)
+        g.replay()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e.record(stream)
+    torch.cuda.synchronize(dev)
+    us = s.elapsed_time(e) * 1e3 / (pool_n * reps)
+    read = nbytes(pool[0].codes) + nbytes(pool[0].scales) + nbytes(pool[0].zeros)
+    return {"us_per_layer": round(us, 3), "gbs": round(read / us / 1e3, 1),
+            "bytes_per_layer": read,
+            "how": "library read-only streaming kernel (16-byte loads, 4 CTAs x 512 threads "
+                   "per SM) over each copy's codes+scales+zeros, CUDA graph of "
+                   f"{pool_n} launches with programmatic dependent launch"}
+
+
+def quantize_bytes(n: int, k: int, bits: int = BITS, group: int = GROUP, sym: bool = SYM) -> int:
+    """Bytes the quantize pass must move: read W (binary16), write codes,
+    scales and (asymmetric) zeros."""
+    return 2 * n * k + n * k * bits // 8 + (n * k // group) * 2 * (1 if sym else 2)
+
+
+def quantize_points(wq, torch, dev, stream, copies: int = 3, reps: int = 10):
+    """wq_quantize on the benchmark layer (W [14336, 4096] binary16, 117 MB),
+    rotating over `copies` different inputs so that the reads come from HBM."""
+    import synth
+    Ws = [synth.weight(N, K, seed=10 + i, device=dev) for i in range(copies)]
+    outs = [wq.quantize(W, bits=BITS, group=GROUP, symmetric=SYM) for W in Ws]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        wq.quantize(Ws[0], bits=BITS, group=GROUP, symmetric=SYM, out=outs[0])
+        stream.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            for W, q in zip(Ws, outs):
+                wq.quantize(W, bits=BITS, group=GROUP, symmetric=SYM, out=q)
+        g.replay()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e.record(stream)
+    torch.cuda.synchronize(dev)
+    us = s.elapsed_time(e) * 1e3 / (copies * reps)
+    b = quantize_bytes(N, K)
+    peak, kind = measured_peaks()
+    return {"us": round(us, 2), "gbs": round(b / us / 1e3, 1), "bytes": b,
+            "frac": round(b / us / 1e3 / peak, 4), "peak_kind": f"{kind} HBM copy",
+            "how": f"CUDA graph over {copies} different W copies (117 MB each)"}
+
+
+def whole_model_quantize(wq, torch, dev, stream, reps: int = 2):
+    """Quantize every matrix of a Llama-8B-shaped model (32 layers x q, k, v,
+    o, gate, up, down = 224 matrices, 6.98e9 binary16 weights, drawn on the
+    GPU with seed 1000 * layer + projection): one CUDA graph of 224 quantize
+    launches, timed as a whole.  The inputs (14 GB) are far larger than the
+    L2."""
+    import synth
+    mats = synth.llama8b_matrices()
+    Ws = [synth.weight(n, k, seed=seed, device=dev) for (_, _, _, n, k, seed) in mats]
+    outs = [wq.quantize(W, bits=BITS, group=GROUP, symmetric=SYM) for W in Ws]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        stream.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            for W, q in zip(Ws, outs):
+                wq.quantize(W, bits=BITS, group=GROUP, symmetric=SYM, out=q)
+        g.replay()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = s.elapsed_time(e) / reps
+    b = sum(quantize_bytes(n, k) for (_, _, _, n, k, _) in mats)
+    params = sum(n * k for (_, _, _, n, k, _) in mats)
+    peak, kind = measured_peaks()
+    del Ws, outs, g
+    torch.cuda.empty_cache()
+    return {"matrices": len(mats), "params": params, "ms": round(ms, 3),
+            "gbs": round(b / ms / 1e6, 1), "bytes": b, "frac": round(b / ms / 1e6 / peak, 4),
+            "peak_kind": f"{kind} HBM copy",
+            "how": "CUDA graph of 224 wq_quantize launches, INT4 asymmetric group 128"}
 
 
 def prefill_points(wq, torch, dev, reps: int = 8):

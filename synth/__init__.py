@@ -29,6 +29,25 @@ LAYER_SHAPES = {          # (K, N) of the Llama-8B projections
 }
 
 
+# The seven projections of one Llama-8B decoder layer, as (name, N, K): the
+# weight of a projection is [N out features, K in features].
+LLAMA8B_PROJECTIONS = (
+    ("q", 4096, 4096), ("k", 1024, 4096), ("v", 1024, 4096), ("o", 4096, 4096),
+    ("gate", 14336, 4096), ("up", 14336, 4096), ("down", 4096, 14336),
+)
+LLAMA8B_LAYERS = 32
+
+
+def llama8b_matrices(layers: int = LLAMA8B_LAYERS):
+    """(layer, projection index, name, N, K, seed) of every quantized matrix
+    of the whole model: 32 layers x 7 projections = 224 matrices,
+    6,979,321,856 weights.  Matrix (layer, j) is drawn with seed
+    1000 * layer + j (outlier columns from seed + 1, as everywhere)."""
+    return [(layer, j, name, n, k, 1000 * layer + j)
+            for layer in range(layers)
+            for j, (name, n, k) in enumerate(LLAMA8B_PROJECTIONS)]
+
+
 def outlier_columns(K: int, seed: int, fraction: float = 0.005) -> torch.Tensor:
     count = int(round(fraction * K))
     g = torch.Generator().manual_seed(seed + 1)

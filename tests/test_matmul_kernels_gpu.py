@@ -1,8 +1,8 @@
-"""The two small-batch kernels behind wq_matmul, each forced in turn, on the
+"""The small-batch kernels behind wq_matmul, each forced in turn, on the
 same seeded inputs against the oracle: the balanced kernel with and without
 its workspace (row tiles summed across CTAs, or whole tiles per SM), under
-programmatic dependent launch, and the cluster-split kernel it replaces for
-M <= 8.  Tolerance as in test_matmul_gpu: |y - y_ref| <= 1e-4 sum|x w|
+programmatic dependent launch, the cluster-split kernel it replaces for
+M <= 8, and the direct-load kernel (4-bit codes, groups of 128, M <= 4).  Tolerance as in test_matmul_gpu: |y - y_ref| <= 1e-4 sum|x w|
 (+ one bfloat16 ulp for bfloat16 out)."""
 import contextlib
 import ctypes
@@ -17,7 +17,7 @@ from tests.gpu_util import check_tolerance, host_bits, oracle_quantize, weight, 
 
 pytestmark = pytest.mark.gpu
 
-AUTO, CLUSTER, BALANCED, BALANCED_SPLIT = 0, 1, 2, 3
+AUTO, CLUSTER, BALANCED, BALANCED_SPLIT, DIRECT = 0, 1, 2, 3, 4
 
 
 @contextlib.contextmanager
@@ -48,7 +48,7 @@ def workspace_clear():
 
 SHAPES = [(1, 14336, 4096), (2, 1000, 4096), (3, 4096, 4096), (5, 1024, 4096), (8, 700, 4096),
           (1, 4096, 14336), (2, 520, 14336), (1, 77, 1024)]
-FORMATS = [(4, 128, False), (4, 64, True), (4, 32, False), (8, 128, False), (8, 64, True),
+FORMATS = [(4, 128, False), (4, 128, True), (4, 64, True), (4, 32, False), (8, 128, False), (8, 64, True),
            (8, 32, False)]
 
 
@@ -84,16 +84,24 @@ def test_balanced_kernel_modes(M, N, K, bits, group, sym):
     with kernel(CLUSTER):
         outs["cluster"] = wq().matmul(Xd, qw)
         outs["cluster_pdl"] = wq().matmul(Xd, qw, static_weights=True)
+    direct = bits == 4 and group == 128 and M <= 4 and K % 512 == 0
+    if direct:
+        with kernel(DIRECT):
+            outs["direct"] = wq().matmul(Xd, qw)
+            outs["direct_pdl"] = wq().matmul(Xd, qw, static_weights=True)
+            outs["direct_bf16"] = wq().matmul(Xd, qw, out_dtype=torch.bfloat16)
     outs["auto"] = wq().matmul(Xd, qw, static_weights=True)
     torch.cuda.synchronize()
     assert wq().get_device_error() == 0
     assert workspace_clear()
     for name, Y in outs.items():
         y = Y.float().cpu().numpy()[ms, ns]
-        check_tolerance(y, y_ref, y_abs, name == "bf16")
+        check_tolerance(y, y_ref, y_abs, name.endswith("bf16"))
     # the same kernel and plan give the same bits with and without PDL
     assert torch.equal(outs["split"], outs["pdl"])
     assert torch.equal(outs["cluster"], outs["cluster_pdl"])
+    if direct:
+        assert torch.equal(outs["direct"], outs["direct_pdl"])
 
 
 def test_back_to_back_static_weights():
@@ -165,3 +173,8 @@ def test_activation_rows_of_wide_dynamic_range(bits, group, sym):
         Y = wq().matmul(X.cuda(), qw)
     torch.cuda.synchronize()
     check_tolerance(Y.cpu().numpy(), y_ref, y_abs, False)
+    if bits == 4 and group == 128:
+        with kernel(DIRECT):
+            Y = wq().matmul(X.cuda(), qw)
+        torch.cuda.synchronize()
+        check_tolerance(Y.cpu().numpy(), y_ref, y_abs, False)

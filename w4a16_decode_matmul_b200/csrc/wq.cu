@@ -13,6 +13,8 @@
 #include "gemv.cuh"
 #include "gemv_sk.cuh"
 #include "gemm.cuh"
+#include "gemv_ld.cuh"
+#include "stream.cuh"
 
 namespace {
 
@@ -400,6 +402,90 @@ struct GemvOp {
   }
 };
 
+// --------------------------------------------------- direct-load kernel
+
+struct LdPlan {
+  wq::ld::Params p;
+  int grid = 1;
+  size_t smem = 0;
+};
+
+// Plan the direct-load kernel: 4-bit codes in groups of 128 with K a
+// multiple of 512 (groups come in pairs; a CTA's scales load in blocks of
+// four), M <= 4; one CTA per SM (at most one per 8-row tile) with the
+// activations, their group sums, the CTA's scales and zeros and the per-warp
+// partial sums of its tiles in shared memory, next to the per-warp rings of
+// codes.
+bool plan_ld(int M, int N, int K, int bits, int group, const DeviceInfo& dev, LdPlan* plan) {
+  using namespace wq::ld;
+  if (bits != 4 || group != kGroup || M < 1 || M > kMaxM || N < 1 || K < 4 * kGroup ||
+      K % (4 * kGroup) != 0)
+    return false;
+  auto round_up = [](size_t a, size_t b) { return (a + b - 1) / b * b; };
+  wq::ld::Params& p = plan->p;
+  p = wq::ld::Params{};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.ngroups = K / kGroup;
+  p.tiles = (N + kTileRows - 1) / kTileRows;
+  plan->grid = std::min(p.tiles, dev.sms);
+  const size_t max_tiles = size_t((p.tiles + plan->grid - 1) / plan->grid);
+  const size_t max_rows = max_tiles * kTileRows;
+  p.xs_row_bytes = uint32_t(K) * 2 + 64;  // rows 64 bytes apart modulo 128: no bank conflicts
+  p.off_sx = uint32_t(round_up(size_t(M) * p.xs_row_bytes, 16));
+  p.off_sz = uint32_t(round_up(p.off_sx + size_t(M) * p.ngroups * 4, 16));
+  p.off_part = uint32_t(round_up(p.off_sz + max_rows * (p.ngroups + 1) * 4, 16));
+  p.off_ring = uint32_t(round_up(p.off_part + max_tiles * kWarps * kTileRows * size_t(M) * 4, 128));
+  plan->smem = p.off_ring + size_t(kWarps) * kDepth * 1024;
+  return plan->smem <= size_t(dev.max_smem_optin);
+}
+
+template <int BITS, bool SYM, int G>
+struct LdOp {
+  static cudaError_t run(LdPlan* plan, const DeviceInfo* dev, cudaStream_t s, bool pdl) {
+    if constexpr (BITS != 4 || G != wq::ld::kGroup) {
+      return cudaErrorInvalidValue;
+    } else {
+      const int M = plan->p.M;
+      if (M == 1) return launch<1>(plan, dev, s, pdl);
+      if (M == 2) return launch<2>(plan, dev, s, pdl);
+      return launch<4>(plan, dev, s, pdl);
+    }
+  }
+
+  template <int MT>
+  static cudaError_t launch(LdPlan* plan, const DeviceInfo* dev, cudaStream_t s, bool pdl) {
+    {
+      auto kernel = &wq::ld::gemv_ld_kernel<SYM, MT>;
+      static int configured[kMaxDevices] = {};
+      int device = 0;
+      cudaGetDevice(&device);
+      if (device < 0 || device >= kMaxDevices) return cudaErrorInvalidDevice;
+      if (!configured[device]) {
+        const cudaError_t e = cudaFuncSetAttribute(
+            kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dev->max_smem_optin);
+        if (e != cudaSuccess) return e;
+        configured[device] = 1;
+      }
+      plan->p.pdl = pdl ? 1 : 0;
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attrs[1];
+      cfg.gridDim = dim3(unsigned(plan->grid));
+      cfg.blockDim = dim3(wq::ld::kThreads);
+      cfg.dynamicSmemBytes = plan->smem;
+      cfg.stream = s;
+      if (pdl) {
+        attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attrs[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attrs;
+        cfg.numAttrs = 1;
+      }
+      return cudaLaunchKernelEx(&cfg, kernel, plan->p);
+    }
+  }
+};
+
 // ------------------------------------------------------- balanced kernel
 
 struct SkPlan {
@@ -413,7 +499,7 @@ struct SkPlan {
 
 // Which small-batch kernel wq_matmul uses: 0 chooses, 1 forces the
 // cluster-split kernel, 2 forces the balanced kernel, 3 forces it with split
-// row tiles (tuning and tests).
+// row tiles, 4 forces the direct-load kernel (tuning and tests).
 int g_kernel_choice = 0;
 
 // Plan the balanced kernel; false if the shape is outside its scope (M <= 8,
@@ -759,17 +845,33 @@ wq_status wq_matmul(const void* X, int64_t M, const void* codes, const void* sca
   const bool have_ws = workspace != nullptr && workspace_bytes >= wq_matmul_workspace_bytes() &&
                        dev.sms <= wq::sk::kWsCtasMax;
 
-  // Kernel choice (measured on B200): the balanced kernel for 8-bit codes,
-  // group 32, and layers with fewer than three waves of row tiles per SM;
-  // the cluster-split kernel otherwise.  Splitting row tiles across CTAs
-  // through the workspace measured slower than whole tiles on every shape
-  // tried (the end-of-kernel gather costs more than the balance gains), so
-  // it is used only when forced through the tuning hook.
   const bool pdl = (flags & WQ_MATMUL_STATIC_WEIGHTS) != 0;
   const int tiles = int((N + 15) / 16);
+  // Kernel choice (measured on B200, back-to-back launches): the direct-load
+  // kernel wherever it applies (4-bit codes, groups of 128, M <= 4, K a
+  // multiple of 512): faster than both others on every Llama-8B layer shape
+  // at M = 1, 2, 4.  Otherwise: the balanced kernel for 8-bit codes, group
+  // 32, and layers with fewer than three waves of row tiles per SM; the
+  // cluster-split kernel otherwise.  Splitting row tiles across CTAs through
+  // the workspace measured slower than whole tiles on every shape tried (the
+  // end-of-kernel gather costs more than the balance gains), so it is used
+  // only when forced through the tuning hook.
+  if (g_kernel_choice == 4 || g_kernel_choice == 0) {
+    LdPlan lp;
+    if (plan_ld(int(M), int(N), int(K), bits, group, dev, &lp)) {
+      lp.p.X = static_cast<const __nv_bfloat16*>(X);
+      lp.p.Y = Y;
+      lp.p.codes = static_cast<const uint8_t*>(codes);
+      lp.p.scales = static_cast<const __half*>(scales);
+      lp.p.zeros = static_cast<const __half*>(zeros);
+      lp.p.y_bf16 = out_dtype == WQ_OUT_BF16;
+      return from_cuda(dispatch_format<LdOp>(bits, symmetric != 0, group, &lp, &dev, s, pdl));
+    }
+    if (g_kernel_choice == 4) return WQ_ERR_UNSUPPORTED;
+  }
   const bool prefer_balanced = bits == 8 || group == 32 || tiles < 3 * dev.sms;
   const bool use_balanced =
-      g_kernel_choice >= 2 || (g_kernel_choice == 0 && prefer_balanced);
+      g_kernel_choice == 2 || g_kernel_choice == 3 || (g_kernel_choice == 0 && prefer_balanced);
   const bool split = have_ws && g_kernel_choice == 3;
   SkPlan sk;
   if (use_balanced &&
@@ -891,8 +993,8 @@ const char* wq_internal_last_cuda_error(void) { return cudaGetErrorName(g_last_c
 // Tuning and test hook, not part of the public ABI: 0 lets wq_matmul choose
 // the small-batch kernel, 1 forces the cluster-split kernel, 2 forces the
 // balanced kernel, 3 forces the balanced kernel with row tiles split across
-// CTAs whenever a workspace is given (2 and 3 return WQ_ERR_UNSUPPORTED
-// where the balanced kernel does not apply).
+// CTAs whenever a workspace is given, 4 forces the direct-load kernel (2, 3
+// and 4 return WQ_ERR_UNSUPPORTED where the forced kernel does not apply).
 void wq_internal_set_kernel(int choice) { g_kernel_choice = choice; }
 
 // Test hook, not part of the public ABI: the balanced kernel's plan for a
@@ -935,6 +1037,25 @@ int wq_internal_plan_gemm(int M, int N, int K, int bits, int group, int symmetri
   return 1;
 }
 
+// Test hook, not part of the public ABI: the direct-load kernel's plan for a
+// device with `sms` SMs and `smem_optin` bytes of shared memory per block,
+// written to out[0..11] (see tests/test_plan_ld.py for the field order).
+// Returns 0 if the shape is outside that kernel's scope.
+int wq_internal_plan_ld(int M, int N, int K, int bits, int group, int sms, int smem_optin,
+                        int64_t* out) {
+  DeviceInfo dev;
+  dev.sms = sms;
+  dev.max_smem_optin = smem_optin;
+  LdPlan plan;
+  if (!plan_ld(M, N, K, bits, group, dev, &plan)) return 0;
+  const wq::ld::Params& p = plan.p;
+  const int64_t v[] = {p.M,      p.N,      p.K,        p.ngroups, p.tiles,
+                       p.xs_row_bytes, p.off_sx, p.off_sz, p.off_part, p.off_ring,
+                       int64_t(plan.smem), plan.grid};
+  for (size_t i = 0; i < sizeof(v) / sizeof(v[0]); ++i) out[i] = v[i];
+  return 1;
+}
+
 // Test hook, not part of the public ABI: the matmul plan for a device with
 // `sms` SMs and `smem_optin` bytes of shared memory per block, written to
 // out[0..27] (see tests/test_plan.py for the field order).  Returns 0 if no
@@ -955,6 +1076,49 @@ int wq_internal_plan_gemv(int M, int N, int K, int bits, int group, int sms, int
                        p.red_bufs, p.row_stride, p.contig};
   for (size_t i = 0; i < sizeof(v) / sizeof(v[0]); ++i) out[i] = v[i];
   return 1;
+}
+
+// Measurement hook, not part of the public ABI: one launch of the read-only
+// streaming kernel over up to three spans (a, b, c; byte counts multiples of
+// 16, pointers 16-byte aligned; a null pointer with size 0 skips a span).  It
+// writes one word per block to `out`, which must hold
+// wq_internal_stream_read_out_bytes() bytes.  `pdl` launches it with
+// programmatic dependent launch, like the fused matmul.
+size_t wq_internal_stream_read_out_bytes(void) {
+  DeviceInfo dev;
+  if (!device_info(&dev)) return 0;
+  return size_t(dev.sms) * wq::stream::kBlocksPerSm * 4;
+}
+
+wq_status wq_internal_stream_read(const void* a, size_t na, const void* b, size_t nb,
+                                  const void* c, size_t nc, void* out, int pdl,
+                                  wq_stream_t stream) {
+  const void* ptrs[3] = {a, b, c};
+  const size_t sizes[3] = {na, nb, nc};
+  for (int i = 0; i < 3; ++i) {
+    if (sizes[i] % 16 != 0 || (sizes[i] != 0 && ptrs[i] == nullptr)) return WQ_ERR_INVALID_ARG;
+    if (ptrs[i] && !aligned16(ptrs[i])) return WQ_ERR_ALIGNMENT;
+  }
+  if (!out) return WQ_ERR_INVALID_ARG;
+  DeviceInfo dev;
+  if (!device_info(&dev)) return WQ_ERR_CUDA;
+  using wq::stream::Span;
+  const Span sa{reinterpret_cast<const uint4*>(a), na / 16};
+  const Span sb{reinterpret_cast<const uint4*>(b), nb / 16};
+  const Span sc{reinterpret_cast<const uint4*>(c), nc / 16};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(dev.sms * wq::stream::kBlocksPerSm));
+  cfg.blockDim = dim3(wq::stream::kThreads);
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  if (pdl) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  return from_cuda(cudaLaunchKernelEx(&cfg, wq::stream::stream_read_kernel, sa, sb, sc,
+                                      reinterpret_cast<uint32_t*>(out)));
 }
 
 }  // extern "C"
