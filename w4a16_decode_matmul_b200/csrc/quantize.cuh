@@ -6,12 +6,15 @@
 // (llminference s08) section 解法 (symmetric: z = 0, s = max|w|/(2^(b-1)-1),
 // codes clipped to [-2^(b-1), 2^(b-1)-1], stored offset by 2^(b-1)).
 //
-// Exactness: weights and the stored scale are binary16 (11-bit
-// significands), so every quotient the method rounds -- w/s and lo/s -- is
-// at least 2^-13 (relative) away from a half-integer unless it is exactly
-// one; an IEEE round-to-nearest binary32 division therefore lands on the
-// same side of every rounding boundary as the exact quotient, and rintf()
-// resolves exact ties to even.  The scale (hi - lo)/qmax is formed in
+// Exactness: the codes are round-half-to-even of the exact quotient w/s.
+// The zero point rounds -lo/s through one IEEE division per group; the
+// codes avoid a division per weight.  With inv = 1/s rounded to nearest,
+// t = w * inv is within 2^-15 of w/s (|w/s| <= 255 because the range
+// contains w and 0), so rintf(t) can differ from the exact rounding only
+// when t lies within 2^-15 of a half-integer h.  In that window (taken as
+// 2^-12) the side is decided exactly: fmaf(-h, s, w) rounds w - h*s once,
+// so its sign is the sign of w/s - h, and it is zero exactly on a tie,
+// which goes to the even neighbour.  The scale (hi - lo)/qmax is formed in
 // binary64 (the difference of two binary16 values is exact there, and the
 // quotient cannot cross a binary16 value), converted with round-up to
 // binary32 and then to binary16; two round-ups compose to one.
@@ -20,6 +23,20 @@
 #include "common.cuh"
 
 namespace wq {
+
+// rint(w / s), ties to even, for s > 0 and |w / s| <= 255 (see the
+// exactness note above); inv is 1/s rounded to nearest.
+__device__ __forceinline__ float rint_quotient(float w, float s, float inv) {
+  const float t = w * inv;
+  float q = rintf(t);
+  const float f = t - q;
+  if (fabsf(fabsf(f) - 0.5f) < 0x1p-12f) {
+    const float h = q + copysignf(0.5f, f);  // the half-integer next to t
+    const float e = fmaf(-h, s, w);          // sign(w/s - h), zero on a tie
+    q = e > 0.f ? h + 0.5f : (e < 0.f ? h - 0.5f : rintf(h));
+  }
+  return q;
+}
 
 // Each lane owns 32 consecutive weights of the flattened [N*K] matrix, so a
 // group of G weights spans G/32 lanes and a warp covers 1024 weights.
@@ -79,11 +96,12 @@ __global__ void __launch_bounds__(256) quantize_kernel(const __half* __restrict_
 
     // Stored scale (binary16, rounded up) and zero point.
     __half s16 = __float2half(1.0f);
-    float s = 1.0f, z = 0.f;
+    float s = 1.0f, inv = 1.0f, z = 0.f;
     if (hi != lo) {
       const double d = __ddiv_rn(double(hi) - double(lo), double(kQmax));
       s16 = __float2half_ru(__double2float_ru(d));
       s = __half2float(s16);
+      inv = __frcp_rn(s);
       if (!SYM) z = fminf(fmaxf(rintf(__fdiv_rn(-lo, s)), 0.f), kQmax);
     }
 
@@ -93,7 +111,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(const __half* __restrict_
     for (int i = 0; i < BITS; ++i) packed[i] = 0;
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-      const float r = rintf(__fdiv_rn(w[i], s));
+      const float r = rint_quotient(w[i], s, inv);
       const float q = SYM ? fminf(fmaxf(r, kQmin), kQmax) + kOffset
                           : fminf(fmaxf(r + z, kQmin), kQmax);
       const uint32_t u = static_cast<uint32_t>(static_cast<int>(q));
