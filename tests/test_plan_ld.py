@@ -48,7 +48,7 @@ def test_plan_layout(lib, M, N, K):
     assert max(shares) <= max_tiles and sum(shares) == tiles
     assert p["xs_row_bytes"] == 2 * K + 64 and p["xs_row_bytes"] % 128 == 64
     regions = [(0, M * p["xs_row_bytes"]), (p["off_sx"], M * ng * 4),
-               (p["off_sz"], max_tiles * TILE_ROWS * (ng + 1) * 4),
+               (p["off_sz"], max_tiles * TILE_ROWS * (ng + 1) * 8),
                (p["off_part"], max_tiles * WARPS * TILE_ROWS * M * 4),
                (p["off_ring"], WARPS * DEPTH * 1024)]
     for (a, n), (b, _) in zip(regions, regions[1:]):

@@ -23,7 +23,7 @@
 //     first DEPTH units are requested before the wait on the previous grid
 //     when the caller promises the weights are static.  The CTA's scales and
 //     zeros (a contiguous block of each tensor) are read once, coalesced,
-//     into shared memory.
+//     into a shared-memory table of binary32 pairs {s, 128 + z}.
 //   * Seen as mma.sync m16n8k16 fragments (lane = 4 g + t), lane L holds row
 //     g of the A operand with g = 2 r + (c / 4), i.e. A row g is (tile row
 //     g / 2, group g % 2 of the pair) and rows g + 8 are tile rows 4 + g / 2.
@@ -71,7 +71,7 @@ struct Params {
   int pdl;                 // weights may be read before the previous grid completes
   uint32_t xs_row_bytes;   // K * 2 + 64: shared-memory bytes per activation row
   uint32_t off_sx;         // [M][ngroups] binary32 group sums
-  uint32_t off_sz;         // [rows of the CTA][ngroups + 1] (scale, zero) binary16 pairs
+  uint32_t off_sz;         // [rows of the CTA][ngroups + 1] {scale, 128 + zero} binary32
   uint32_t off_part;       // [tiles per CTA][kWarps][8][M] binary32 partials
   uint32_t off_ring;       // [kWarps][kDepth][2][32 lanes][16 bytes] codes ring
 };
@@ -101,7 +101,7 @@ __device__ __forceinline__ uint2 ldg_stream64(const void* p) {
 // The fetch side of a warp's units: the byte offset of this lane's 16 bytes
 // of tile row r in the codes, and whether rows r and r + 4 exist.
 struct FetchWalk {
-  size_t ofs;
+  const uint8_t* ptr;  // this lane's 16 bytes of tile row r
   int pair, left;
   bool ok0, ok1;
   int row0;
@@ -111,10 +111,10 @@ struct FetchWalk {
   }
   __device__ __forceinline__ void next(int pairs, size_t row_bytes, int N) {
     --left;
-    ofs += kUnitBytes;
+    ptr += kUnitBytes;
     if (++pair == pairs) {  // next tile: 8 rows down, back to the first pair
       pair = 0;
-      ofs += 7 * row_bytes;
+      ptr += 7 * row_bytes;
       row0 += kTileRows;
       set_rows(N);
     }
@@ -125,8 +125,8 @@ struct FetchWalk {
 // r + 4 at dst + 512); rows past N are zero-filled without reading.
 __device__ __forceinline__ void load_unit(const uint8_t* codes, const FetchWalk& f,
                                           size_t row_bytes, uint32_t dst) {
-  cp_async16(dst, f.ok0 ? codes + f.ofs : codes, f.ok0);
-  cp_async16(dst + 512, f.ok1 ? codes + f.ofs + 4 * row_bytes : codes, f.ok1);
+  cp_async16(dst, f.ok0 ? f.ptr : codes, f.ok0);
+  cp_async16(dst + 512, f.ok1 ? f.ptr + 4 * row_bytes : codes, f.ok1);
 }
 
 // Units in order: tile-major, pair-minor.
@@ -162,7 +162,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_ld_kernel(const Params p) {
   fetch.pair = use.pair;
   fetch.left = use.left;
   fetch.row0 = use.tile * kTileRows + r;
-  fetch.ofs = size_t(fetch.row0) * row_bytes + size_t(use.pair) * kUnitBytes + size_t(c) * 16;
+  fetch.ptr = p.codes + size_t(fetch.row0) * row_bytes + size_t(use.pair) * kUnitBytes +
+              size_t(c) * 16;
   fetch.set_rows(p.N);
   // this lane's 16 bytes of slot 0 (row r); slot j at + 1024 j
   const uint32_t ring = smem_addr(smem) + p.off_ring + uint32_t(warp * kDepth * 1024 + lane * 16);
@@ -207,9 +208,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_ld_kernel(const Params p) {
   }
 
   float* sx = reinterpret_cast<float*>(smem + p.off_sx);
-  uint32_t* sz = reinterpret_cast<uint32_t*>(smem + p.off_sz);
+  float2* sz = reinterpret_cast<float2*>(smem + p.off_sz);
   float* part = reinterpret_cast<float*>(smem + p.off_part);
-  const int sz_stride = ng + 1;  // words per row: rows land on different banks
+  const int sz_stride = ng + 1;  // entries per row: rows land on different banks
   {
     // activations, permuted, and their group sums
     const int total8 = p.M * p.K / 8;  // a multiple of 16: groups of 128 never straddle
@@ -238,15 +239,20 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_ld_kernel(const Params p) {
       for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
       if (ok && (threadIdx.x & 15) == 0) sx[(8 * i) / kGroup] = sum;  // [n][gi] flattened
     }
-    // scales and zeros as (scale, zero) pairs: the blocks held in registers,
-    // then any further blocks of a large CTA share
+    // scales and zeros as {s, 128 + z} (symmetric: 128 + 8): the blocks held
+    // in registers, then any further blocks of a large CTA share
     auto store_meta = [&](int i, uint2 a, uint2 z) {
       const int e = 4 * i, row = e / ng, gi = e - row * ng;
-      uint32_t* d = sz + row * sz_stride + gi;
-      d[0] = __byte_perm(a.x, z.x, 0x5410);
-      d[1] = __byte_perm(a.x, z.x, 0x7632);
-      d[2] = __byte_perm(a.y, z.y, 0x5410);
-      d[3] = __byte_perm(a.y, z.y, 0x7632);
+      float2* d = sz + row * sz_stride + gi;
+      const uint32_t sw[2] = {a.x, a.y}, zw[2] = {z.x, z.y};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t sk = (sw[k >> 1] >> (16 * (k & 1))) & 0xFFFFu;
+        const uint32_t zk = (zw[k >> 1] >> (16 * (k & 1))) & 0xFFFFu;
+        const float bias =
+            SYM ? 136.f : 128.f + __half2float(__ushort_as_half(static_cast<unsigned short>(zk)));
+        d[k] = make_float2(__half2float(__ushort_as_half(static_cast<unsigned short>(sk))), bias);
+      }
     };
 #pragma unroll
     for (int j = 0; j < kMetaRegs; ++j) {
@@ -279,6 +285,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_ld_kernel(const Params p) {
   const int rr0 = g >> 1, rr1 = rr0 + 4;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   int cur_tile = use.tile;
+  // this lane's rows of the {s, 128 + z} table for the current tile, and its
+  // tokens' group sums
+  const float2* sz0 = sz + ((cur_tile - tb0) * kTileRows + rr0) * sz_stride;
+  const float* sx0 = sx + m0 * ng;
+  const float* sx1 = sx + m1 * ng;
 
   // Lanes L and L ^ 6 own the same outputs for the two groups of a pair:
   // their sums are added (group A's lane first) and group A's lane stores.
@@ -307,6 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_ld_kernel(const Params p) {
         if (use.tile != cur_tile) {
           flush();
           cur_tile = use.tile;
+          sz0 = sz + ((cur_tile - tb0) * kTileRows + rr0) * sz_stride;
         }
         cp_async_wait<kDepth - 1>();  // this unit's copies (issued by this lane) landed
         const uint4 c0 = lds128(ring + uint32_t(j) * 1024);
@@ -336,26 +348,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_ld_kernel(const Params p) {
         if (owner) {
           // y += s * (C - (128 + z) * Sx), per row, in binary32
           const int gi = 2 * pair + hh;
-          const int lrow = (cur_tile - tb0) * kTileRows;
-          const uint32_t e0 = sz[(lrow + rr0) * sz_stride + gi];
-          const uint32_t e1 = sz[(lrow + rr1) * sz_stride + gi];
-          const float s0 = __half2float(__ushort_as_half(static_cast<unsigned short>(e0)));
-          const float s1 = __half2float(__ushort_as_half(static_cast<unsigned short>(e1)));
-          const float b0 = SYM ? 136.f
-                               : 128.f + __half2float(__ushort_as_half(
-                                             static_cast<unsigned short>(e0 >> 16)));
-          const float b1 = SYM ? 136.f
-                               : 128.f + __half2float(__ushort_as_half(
-                                             static_cast<unsigned short>(e1 >> 16)));
+          const float2 e0 = sz0[gi];                       // tile row rr0
+          const float2 e1 = sz0[4 * sz_stride + gi];       // tile row rr0 + 4
           if (use0) {
-            const float x = sx[m0 * ng + gi];
-            acc[0] = fmaf(s0, fmaf(-b0, x, d[0]), acc[0]);
-            acc[2] = fmaf(s1, fmaf(-b1, x, d[2]), acc[2]);
+            const float x = sx0[gi];
+            acc[0] = fmaf(e0.x, fmaf(-e0.y, x, d[0]), acc[0]);
+            acc[2] = fmaf(e1.x, fmaf(-e1.y, x, d[2]), acc[2]);
           }
           if (use1) {
-            const float x = sx[m1 * ng + gi];
-            acc[1] = fmaf(s0, fmaf(-b0, x, d[1]), acc[1]);
-            acc[3] = fmaf(s1, fmaf(-b1, x, d[3]), acc[3]);
+            const float x = sx1[gi];
+            acc[1] = fmaf(e0.x, fmaf(-e0.y, x, d[1]), acc[1]);
+            acc[3] = fmaf(e1.x, fmaf(-e1.y, x, d[3]), acc[3]);
           }
         }
         use.next(pairs);

@@ -435,7 +435,7 @@ bool plan_ld(int M, int N, int K, int bits, int group, const DeviceInfo& dev, Ld
   p.xs_row_bytes = uint32_t(K) * 2 + 64;  // rows 64 bytes apart modulo 128: no bank conflicts
   p.off_sx = uint32_t(round_up(size_t(M) * p.xs_row_bytes, 16));
   p.off_sz = uint32_t(round_up(p.off_sx + size_t(M) * p.ngroups * 4, 16));
-  p.off_part = uint32_t(round_up(p.off_sz + max_rows * (p.ngroups + 1) * 4, 16));
+  p.off_part = uint32_t(round_up(p.off_sz + max_rows * (p.ngroups + 1) * 8, 16));
   p.off_ring = uint32_t(round_up(p.off_part + max_tiles * kWarps * kTileRows * size_t(M) * 4, 128));
   plan->smem = p.off_ring + size_t(kWarps) * kDepth * 1024;
   return plan->smem <= size_t(dev.max_smem_optin);
