@@ -11,6 +11,9 @@ Two parts:
   and binary16 integer zeros out; dequantization and the matmul in double.
 * ``oracle.paper``: the pages' own Python-float semantics ("paper mode"),
   used for the worked examples.
+* the nested-superblock quantizer (page 2's Q4_K figure; 4.5 bits per
+  weight) in ``oracle.c``, pinned by ``tests/test_oracle_q4k.py``.
+* ``oracle.snr_table``: information-only error and traffic tables.
 
 Every function states the passage it follows in its docstring or in the C
 source.  Parity of the storage-mode quantizer is pinned by exact-rational
@@ -69,6 +72,10 @@ class Oracle:
         lib.oracle_matmul_at.restype = None
         lib.oracle_matmul_dense_bf16.argtypes = [vp, i64, vp, i64, i64, vp]
         lib.oracle_matmul_dense_bf16.restype = None
+        lib.oracle_q4k_quantize.argtypes = [vp, i64, i64, vp]
+        lib.oracle_q4k_quantize.restype = None
+        lib.oracle_q4k_dequantize.argtypes = [vp, i64, i64, vp]
+        lib.oracle_q4k_dequantize.restype = None
         lib.oracle_half_to_double.argtypes = [ctypes.c_uint16]
         lib.oracle_half_to_double.restype = ctypes.c_double
         lib.oracle_half_round_up.argtypes = [ctypes.c_double]
@@ -115,6 +122,37 @@ class Oracle:
         self.lib.oracle_dequantize(_p(codes), _p(scales), _p(zp), N, K, bits, group,
                                    int(bool(symmetric)), _p(out))
         return out
+
+    # -- nested superblocks -----------------------------------------------
+    Q4K_BLOCK_BYTES = 144  # per 256 weights: 4.5 bits per weight
+
+    def q4k_quantize(self, W_half_bits: np.ndarray) -> np.ndarray:
+        """Superblock quantizer (page 2 "量化", the Q4_K figure; the reading is
+        stated in oracle.c).  ``W_half_bits`` is uint16 [N, K], K a multiple of
+        256.  Returns the blocks, uint8 [N, K/256 * 144]."""
+        W = np.ascontiguousarray(W_half_bits, dtype=np.uint16)
+        N, K = W.shape
+        assert K % 256 == 0
+        blocks = np.zeros((N, K // 256 * self.Q4K_BLOCK_BYTES), dtype=np.uint8)
+        self.lib.oracle_q4k_quantize(_p(W), N, K, _p(blocks))
+        return blocks
+
+    def q4k_dequantize(self, blocks: np.ndarray, N: int, K: int) -> np.ndarray:
+        """What = S_j q - M_j in double, [N, K], from the blocks' bytes."""
+        blocks = np.ascontiguousarray(blocks, dtype=np.uint8)
+        assert blocks.shape == (N, K // 256 * self.Q4K_BLOCK_BYTES)
+        out = np.empty((N, K), dtype=np.float64)
+        self.lib.oracle_q4k_dequantize(_p(blocks), N, K, _p(out))
+        return out
+
+    def q4k_matmul(self, X_bf16_bits, blocks: np.ndarray, N: int, K: int):
+        """``(Y, Yabs)`` for superblock weights: Y = X What^T and sum |x w|
+        per output, in double."""
+        X = np.asarray([self.lib.oracle_bf16_to_double(int(v)) for v in
+                        np.asarray(X_bf16_bits, dtype=np.uint16).ravel()],
+                       dtype=np.float64).reshape(-1, K)
+        Wh = self.q4k_dequantize(blocks, N, K)
+        return X @ Wh.T, np.abs(X) @ np.abs(Wh).T
 
     # -- matmul ------------------------------------------------------------
     def matmul(self, X_bf16_bits, codes, scales, zeros, N: int, K: int, bits: int,

@@ -307,6 +307,115 @@ void oracle_matmul_dense_bf16(const uint16_t *X, int64_t M, const uint16_t *B,
 }
 
 /* Exposed for the tests' independent checks of the decoders. */
+/* ---- nested superblocks (Q4_K-style), 4.5 bits per weight ---------------
+ *
+ * [P2] "量化", the Q4_K superblock figure: 256 weights in 8 subblocks of 32;
+ * every subblock has a 6-bit scale and a 6-bit minimum, themselves quantized
+ * against a binary16 super-scale d and super-minimum dmin; 4-bit codes;
+ * 4.5 bits per weight.  The page fixes only the nesting and the bit counts.
+ * The plain reading taken here (listed in the design notes):
+ *   subblock j:  lo = min(0, min w), hi = max(0, max w)  (P1's range),
+ *                s_j = (hi - lo) / 15,  m_j = -lo;
+ *   d    = smallest binary16 >= max_j s_j / 63  (0 when every s_j is 0),
+ *   dmin = smallest binary16 >= max_j m_j / 63  (0 when every m_j is 0);
+ *   sc_j = clamp(round(s_j / d), 1, 63)     (1 when d = 0),
+ *   mq_j = clamp(round(m_j / dmin), 0, 63)  (0 when dmin = 0);
+ *   S_j = d sc_j,  M_j = dmin mq_j  (exact);
+ *   q = clamp(round((w + M_j) / S_j), 0, 15)  (0 when S_j = 0);
+ *   w^ = S_j q - M_j.
+ * Every rounding is round-half-to-even of the exact quotient: the operands
+ * are binary16 values and products of them with small integers, so the
+ * double-precision quotients land on the right side of every half-integer
+ * and exact ties stay exact.
+ * Block layout (144 bytes): d (binary16, little-endian), dmin, 12 bytes
+ * holding sc_0..sc_7 then mq_0..mq_7 as 6-bit fields, least significant bit
+ * first (field f in bits 6f .. 6f+5 of the 96-bit little-endian value), then
+ * 128 bytes of codes (byte i: weight 2i in the low nibble, 2i+1 in the high).
+ * Blocks run along K: block b of row n covers k = 256 b .. 256 b + 255, and
+ * row n's blocks are contiguous (K/256 blocks per row). */
+void oracle_q4k_quantize(const uint16_t *W, int64_t N, int64_t K, uint8_t *blocks)
+{
+    const int64_t nb = K / 256;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; n++) {
+        for (int64_t b = 0; b < nb; b++) {
+            const uint16_t *w = W + n * K + b * 256;
+            uint8_t *blk = blocks + (n * nb + b) * 144;
+            double s[8], m[8], smax = 0.0, mmax = 0.0;
+            for (int j = 0; j < 8; j++) {
+                double lo = 0.0, hi = 0.0;
+                for (int i = 0; i < 32; i++) {
+                    double v = half_bits_to_double(w[32 * j + i]);
+                    if (v < lo) lo = v;
+                    if (v > hi) hi = v;
+                }
+                s[j] = (hi - lo) / 15.0;
+                m[j] = -lo;
+                if (s[j] > smax) smax = s[j];
+                if (m[j] > mmax) mmax = m[j];
+            }
+            uint16_t d16 = smax > 0.0 ? half_round_up_positive(smax / 63.0) : 0;
+            uint16_t dm16 = mmax > 0.0 ? half_round_up_positive(mmax / 63.0) : 0;
+            double d = half_bits_to_double(d16), dmin = half_bits_to_double(dm16);
+            int sc[8], mq[8];
+            for (int j = 0; j < 8; j++) {
+                sc[j] = d > 0.0 ? (int)clampd(nearbyint(s[j] / d), 1.0, 63.0) : 1;
+                mq[j] = dmin > 0.0 ? (int)clampd(nearbyint(m[j] / dmin), 0.0, 63.0) : 0;
+            }
+            memset(blk, 0, 144);
+            blk[0] = (uint8_t)(d16 & 0xff);
+            blk[1] = (uint8_t)(d16 >> 8);
+            blk[2] = (uint8_t)(dm16 & 0xff);
+            blk[3] = (uint8_t)(dm16 >> 8);
+            for (int f = 0; f < 16; f++) {
+                int v = f < 8 ? sc[f] : mq[f - 8];
+                for (int bit = 0; bit < 6; bit++) {
+                    if ((v >> bit) & 1) {
+                        int pos = 6 * f + bit;
+                        blk[4 + pos / 8] |= (uint8_t)(1u << (pos % 8));
+                    }
+                }
+            }
+            for (int k = 0; k < 256; k++) {
+                int j = k / 32;
+                double S = d * sc[j], M = dmin * mq[j];
+                double v = half_bits_to_double(w[k]);
+                int q = S > 0.0 ? (int)clampd(nearbyint((v + M) / S), 0.0, 15.0) : 0;
+                blk[16 + k / 2] |= (uint8_t)((k & 1) ? (q << 4) : q);
+            }
+        }
+    }
+}
+
+/* w^ = S_j q - M_j for every weight of the blocks written by
+ * oracle_q4k_quantize (fields read back from the bytes); out is [N][K]. */
+void oracle_q4k_dequantize(const uint8_t *blocks, int64_t N, int64_t K, double *out)
+{
+    const int64_t nb = K / 256;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; n++) {
+        for (int64_t b = 0; b < nb; b++) {
+            const uint8_t *blk = blocks + (n * nb + b) * 144;
+            double d = half_bits_to_double((uint16_t)(blk[0] | (blk[1] << 8)));
+            double dmin = half_bits_to_double((uint16_t)(blk[2] | (blk[3] << 8)));
+            int field[16];
+            for (int f = 0; f < 16; f++) {
+                int v = 0;
+                for (int bit = 0; bit < 6; bit++) {
+                    int pos = 6 * f + bit;
+                    v |= ((blk[4 + pos / 8] >> (pos % 8)) & 1) << bit;
+                }
+                field[f] = v;
+            }
+            for (int k = 0; k < 256; k++) {
+                int j = k / 32;
+                int q = (blk[16 + k / 2] >> ((k & 1) * 4)) & 0x0f;
+                out[n * K + b * 256 + k] = d * field[j] * q - dmin * field[8 + j];
+            }
+        }
+    }
+}
+
 double oracle_half_to_double(uint16_t h) { return half_bits_to_double(h); }
 uint16_t oracle_half_round_up(double x) { return half_round_up_positive(x); }
 double oracle_bf16_to_double(uint16_t b) { return bf16_bits_to_double(b); }
