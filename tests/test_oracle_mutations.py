@@ -2,7 +2,6 @@
 catch every one of them (CPU only; the planted copies are compiled into a
 temporary directory and never touch the real oracle)."""
 import os
-import shutil
 
 import pytest
 
@@ -86,5 +85,7 @@ def test_planted_mistake_is_caught(tmp_path, name, old, new):
         except AssertionError:
             caught.append(check_name)
             break
+    # the planted library is left in place: deleting it would let a later
+    # build reuse its inode, and the dynamic loader would hand back this
+    # library instead of the new one
     assert caught, f"no pin caught the planted mistake '{name}'"
-    shutil.rmtree(tmp_path, ignore_errors=True)
