@@ -42,8 +42,16 @@ WORKLOAD = ("decode GEMV, Llama-8B gate/up layer: M=1, K=4096, N=14336, INT4 asy
             "group 128, fp16 scale+zero, bf16 X, fp32 Y")
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "gemv_w4a16_m1_k4096_n14336.json")
-KERNEL_SOURCES = [os.path.join(ROOT, "w4a16_decode_matmul_b200", "csrc", f)
-                  for f in ("gemv_ld.cuh", "unpack.cuh", "common.cuh", "wq.cu")]
+CSRC = os.path.join(ROOT, "w4a16_decode_matmul_b200", "csrc")
+# What decides the timed kernel: its device code, the host plan and launch of
+# it, and the matmul entry point that chooses it.
+KERNEL_SOURCES = [os.path.join(CSRC, f) for f in ("gemv_ld.cuh", "unpack.cuh", "common.cuh")]
+KERNEL_HOST_SECTIONS = [
+    ("// --------------------------------------------------- direct-load kernel",
+     "// ------------------------------------------------------- balanced kernel"),
+    ("wq_status wq_matmul(const void* X, int64_t M,",
+     "// ------------------------------------------------------ no-allocation entry"),
+]
 
 
 def algorithmic_bytes(m: int = M, n: int = N, k: int = K, bits: int = BITS,
@@ -55,9 +63,15 @@ def algorithmic_bytes(m: int = M, n: int = N, k: int = K, bits: int = BITS,
 
 
 def kernel_source_hash() -> str:
+    """Hash of the sources that decide the timed kernel (device headers, and
+    the sections of wq.cu that plan, choose and launch it)."""
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
         h.update(open(f, "rb").read())
+    host = open(os.path.join(CSRC, "wq.cu"), encoding="utf-8").read()
+    for start, end in KERNEL_HOST_SECTIONS:
+        i = host.index(start)
+        h.update(host[i:host.index(end, i)].encode("utf-8"))
     return h.hexdigest()[:16]
 
 
