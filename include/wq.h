@@ -168,6 +168,45 @@ wq_status wq_matmul_noalloc(const void *X, int64_t M, const void *codes, const v
                             int symmetric, void *Y, int out_dtype, unsigned int flags,
                             wq_stream_t stream);
 
+/* ---- nested superblocks, 4.5 bits per weight -----------------------------
+ * "量化" (llminference s08), the Q4_K superblock figure: 256 weights in 8
+ * sub-blocks of 32, a 6-bit scale and a 6-bit minimum per sub-block
+ * quantized against a binary16 super-scale d and super-minimum dmin, 4-bit
+ * codes.  The page fixes the nesting and the bit counts only; this format
+ * is the library's reading (not GGUF-compatible):
+ *   sub-block j: lo = min(0, min w), hi = max(0, max w) ("vLLM 量化与推测
+ *   解码" section 1's range); s_j = (hi - lo)/15; m_j = -lo;
+ *   d = smallest binary16 >= max s_j / 63, dmin likewise for m_j (0 when the
+ *   maximum is 0); sc_j = clamp(round(s_j/d), 1, 63) (1 when d = 0);
+ *   mq_j = clamp(round(m_j/dmin), 0, 63) (0 when dmin = 0);
+ *   q = clamp(round((w + M_j)/S_j), 0, 15) with S_j = d sc_j, M_j = dmin mq_j
+ *   (0 when S_j = 0); reconstruction w^ = S_j q - M_j.
+ * Every rounding is half-to-even of the exact value.
+ * Layout: row-major [N][K/256] blocks of 144 bytes: d, dmin (binary16,
+ * little-endian), 12 bytes of sixteen 6-bit fields (sc_0..7 then mq_0..7,
+ * least significant bit first), 128 bytes of codes (byte i holds weight 2i
+ * in its low nibble, 2i+1 in its high nibble).  K a multiple of 256.
+ * Errors, checked on the host before any launch: WQ_ERR_INVALID_ARG for a
+ * size outside that scope, M outside 1..8, a null pointer or an unknown
+ * out_dtype; WQ_ERR_ALIGNMENT for a pointer not 16-byte aligned. */
+
+/* Bytes of the blocks of an [N][K] matrix: N*(K/256)*144 (4.5 bits per
+ * weight); 0 for invalid sizes. */
+size_t wq_q4k_bytes(int64_t N, int64_t K);
+
+/* Quantize W [N][K] binary16 into blocks (wq_q4k_bytes(N, K) bytes, 16-byte
+ * aligned, caller-owned).  Bit-exact with the definition above. */
+wq_status wq_q4k_quantize(const void *W, int64_t N, int64_t K, void *blocks,
+                          wq_stream_t stream);
+
+/* Y [M][N] = X [M][K] (bfloat16) * What^T for superblock weights, 1 <= M <=
+ * 8, binary32 accumulation (per sub-block: d sc (sum x q) - dmin mq (sum x));
+ * Y binary32 or bfloat16 (out_dtype as for wq_matmul).  The full-precision
+ * weights are never written.  Pointers 16-byte aligned; nothing is
+ * allocated; the call is enqueued on `stream`. */
+wq_status wq_q4k_matmul(const void *X, int64_t M, const void *blocks, int64_t N, int64_t K,
+                        void *Y, int out_dtype, wq_stream_t stream);
+
 /* Read and clear the device status word (WQ_OK if no kernel recorded an
  * error).  Synchronizes `stream` first. */
 wq_status wq_get_device_error(wq_stream_t stream);

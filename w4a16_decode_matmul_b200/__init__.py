@@ -66,6 +66,12 @@ def _load() -> ctypes.CDLL:
     lib.wq_matmul_noalloc.restype = i32
     lib.wq_matmul_noalloc_scratch_bytes.argtypes = []
     lib.wq_matmul_noalloc_scratch_bytes.restype = sz
+    lib.wq_q4k_bytes.argtypes = [i64, i64]
+    lib.wq_q4k_bytes.restype = sz
+    lib.wq_q4k_quantize.argtypes = [vp, i64, i64, vp, vp]
+    lib.wq_q4k_quantize.restype = i32
+    lib.wq_q4k_matmul.argtypes = [vp, i64, vp, i64, i64, vp, i32, vp]
+    lib.wq_q4k_matmul.restype = i32
     lib.wq_get_device_error.argtypes = [vp]
     lib.wq_get_device_error.restype = i32
     lib.wq_status_string.argtypes = [i32]
@@ -224,6 +230,45 @@ def matmul(X: torch.Tensor, qw: QuantizedWeight, out_dtype: torch.dtype = torch.
         out.copy_(Yd, non_blocking=True)
         return out
     return Yd.cpu()
+
+
+def q4k_bytes(N: int, K: int) -> int:
+    """``wq_q4k_bytes``: bytes of the superblocks of an [N, K] matrix."""
+    return int(lib.wq_q4k_bytes(N, K))
+
+
+def q4k_quantize(W: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """``wq_q4k_quantize``: W [N, K] float16 on the GPU -> uint8 blocks
+    [N, K/256 * 144] (nested superblocks, 4.5 bits per weight)."""
+    if W.dtype != torch.float16 or W.dim() != 2:
+        raise ValueError("W must be a 2-D float16 tensor")
+    N, K = W.shape
+    nb = q4k_bytes(N, K)
+    if nb == 0:
+        raise WQError(1, "wq_q4k_quantize")
+    if out is None:
+        out = torch.empty((N, nb // N), dtype=torch.uint8, device=W.device)
+    _require_cuda(W, out)
+    _check(lib.wq_q4k_quantize(_ptr(W), N, K, _ptr(out), _stream(W.device)), "wq_q4k_quantize")
+    return out
+
+
+def q4k_matmul(X: torch.Tensor, blocks: torch.Tensor, N: int, K: int,
+               out_dtype: torch.dtype = torch.float32,
+               out: torch.Tensor | None = None) -> torch.Tensor:
+    """``wq_q4k_matmul``: Y [M, N] = X [M, K] (bfloat16, M <= 8) times What^T
+    for superblock weights; X, blocks and Y on the GPU."""
+    if X.dtype != torch.bfloat16 or X.dim() != 2 or X.shape[1] != K:
+        raise ValueError("X must be a 2-D bfloat16 tensor [M, K]")
+    if out_dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("out_dtype must be float32 or bfloat16")
+    M = X.shape[0]
+    Y = out if out is not None else torch.empty((M, N), dtype=out_dtype, device=X.device)
+    _require_cuda(X, blocks, Y)
+    _check(lib.wq_q4k_matmul(_ptr(X), M, _ptr(blocks), N, K, _ptr(Y),
+                             WQ_OUT_BF16 if Y.dtype == torch.bfloat16 else WQ_OUT_F32,
+                             _stream(X.device)), "wq_q4k_matmul")
+    return Y
 
 
 def matmul_noalloc(X: torch.Tensor, qw: QuantizedWeight, out_dtype: torch.dtype = torch.float32,

@@ -15,6 +15,7 @@
 #include "gemm.cuh"
 #include "gemv_ld.cuh"
 #include "stream.cuh"
+#include "q4k.cuh"
 
 namespace {
 
@@ -1119,6 +1120,58 @@ wq_status wq_internal_stream_read(const void* a, size_t na, const void* b, size_
   }
   return from_cuda(cudaLaunchKernelEx(&cfg, wq::stream::stream_read_kernel, sa, sb, sc,
                                       reinterpret_cast<uint32_t*>(out)));
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------ nested superblocks
+
+extern "C" {
+
+size_t wq_q4k_bytes(int64_t N, int64_t K) {
+  if (N < 1 || K < wq::q4k::kBlockWeights || K % wq::q4k::kBlockWeights != 0 ||
+      N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
+    return 0;
+  return size_t(N) * size_t(K / wq::q4k::kBlockWeights) * wq::q4k::kBlockBytes;
+}
+
+wq_status wq_q4k_quantize(const void* W, int64_t N, int64_t K, void* blocks,
+                          wq_stream_t stream) {
+  if (wq_q4k_bytes(N, K) == 0 || !W || !blocks) return WQ_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(blocks)) return WQ_ERR_ALIGNMENT;
+  DeviceInfo dev;
+  if (!device_info(&dev)) return WQ_ERR_CUDA;
+  const int64_t nblocks = N * (K / wq::q4k::kBlockWeights);
+  const int64_t grid = std::max<int64_t>(1, std::min<int64_t>((nblocks + 7) / 8,
+                                                               int64_t(dev.sms) * 16));
+  wq::q4k::quantize_kernel<<<unsigned(grid), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __half*>(W), nblocks, static_cast<uint8_t*>(blocks));
+  return from_cuda(cudaGetLastError());
+}
+
+wq_status wq_q4k_matmul(const void* X, int64_t M, const void* blocks, int64_t N, int64_t K,
+                        void* Y, int out_dtype, wq_stream_t stream) {
+  if (wq_q4k_bytes(N, K) == 0 || M < 1 || M > 8 || !X || !blocks || !Y)
+    return WQ_ERR_INVALID_ARG;
+  if (out_dtype != WQ_OUT_F32 && out_dtype != WQ_OUT_BF16) return WQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(blocks) || !aligned16(Y)) return WQ_ERR_ALIGNMENT;
+  DeviceInfo dev;
+  if (!device_info(&dev)) return WQ_ERR_CUDA;
+  const int64_t grid = std::max<int64_t>(1, std::min<int64_t>((N + 7) / 8, int64_t(dev.sms) * 8));
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const auto* x = static_cast<const __nv_bfloat16*>(X);
+  const auto* b = static_cast<const uint8_t*>(blocks);
+  const int yb = out_dtype == WQ_OUT_BF16;
+  const unsigned g = unsigned(grid);
+  if (M == 1)
+    wq::q4k::matmul_kernel<1><<<g, 256, 0, s>>>(x, int(M), b, int(N), int(K), Y, yb);
+  else if (M == 2)
+    wq::q4k::matmul_kernel<2><<<g, 256, 0, s>>>(x, int(M), b, int(N), int(K), Y, yb);
+  else if (M <= 4)
+    wq::q4k::matmul_kernel<4><<<g, 256, 0, s>>>(x, int(M), b, int(N), int(K), Y, yb);
+  else
+    wq::q4k::matmul_kernel<8><<<g, 256, 0, s>>>(x, int(M), b, int(N), int(K), Y, yb);
+  return from_cuda(cudaGetLastError());
 }
 
 }  // extern "C"
