@@ -17,7 +17,8 @@
 // dequantized weight tile):
 //   warp 0      TMA: the 128 x 64 activation tile (128-byte swizzle) and the
 //               128 rows x 64 codes; once per tile the tile's scales/zeros;
-//   warps 2-9   dequantize: half a row of codes per thread -> 32 bfloat16
+//   warps 2-9   dequantize: half a row of codes per thread (the two halves of
+//               a row on adjacent lanes) -> 32 bfloat16
 //               (q - z) written in the same swizzled K-major layout, then an
 //               async-proxy fence and an arrive;
 //   warp 1      one thread issues tcgen05.mma (M=128, N=128, K=16, bfloat16
@@ -319,18 +320,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < kEpilogueWarp0) {
     // ------------------------------------------------------------ dequantize
+    // Two lanes per row, side by side: a warp's code reads are contiguous and
+    // the swizzled tile writes stay free of bank conflicts.
     const int dt = threadIdx.x - kDequantWarp0 * 32;  // 0..255
-    const int r = dt & (kBN - 1);                     // row of the W tile
-    const int part = dt >> 7;                         // 16-byte chunks 4*part .. 4*part+3
+    const int r = dt >> 1;                            // row of the W tile
+    const int part = dt & 1;                          // 16-byte chunks 4*part .. 4*part+3
     const bool have_meta = wait(kBarMeta, 0);
     const __half* zrow = reinterpret_cast<const __half*>(smem + p.off_meta_z) + r * p.ngroups;
+    int zc_group = -1;  // the zero point is read once per group
+    float zc = float(1 << (BITS - 1));
     for (int kb = 0; kb < nkb && have_meta; ++kb) {
       const int s = kb % kStages;
       const uint32_t ph = uint32_t(kb / kStages) & 1u;
       // codes landed, and the previous MMAs of this slot are done with B
       if (!wait(kBarLdFull + s, ph) || !wait(kBarEmpty + s, ph ^ 1u)) break;
       const int gi = kb / kKbPerGroup;
-      const float zc = SYM ? float(1 << (BITS - 1)) : __half2float(zrow[gi]);
+      if (!SYM && gi != zc_group) {
+        zc = __half2float(zrow[gi]);
+        zc_group = gi;
+      }
       const uint8_t* crow = smem + p.off_codes + s * p.codes_stage_bytes + r * kCodesRowBytes;
       uint8_t* brow = smem + p.off_b + s * kTileBytes + r * 128;
       if constexpr (BITS == 4) {
