@@ -20,6 +20,10 @@
  *               accumulated in higher precision; "量化" (llminference s08)
  *               section 实现: dequantize inside the accumulation, never write
  *               full-precision weights back to memory).
+ *   q4k_*       the same two operations for nested superblocks of 256
+ *               weights at 4.5 bits per weight ("量化" (llminference s08),
+ *               the Q4_K superblock figure); the format is given with those
+ *               entry points below.
  *
  * Numerics (fixed where the pages leave them open):
  *   - round() is round-half-to-even; the arithmetic that decides each code
