@@ -57,6 +57,34 @@ def test_payload_sizes_match_page_1(lib):
     assert lib.wq_meta_elems(4, 100, 32) == 0
 
 
+def test_superblock_sizes(lib):
+    """Page 2's superblock budget: 4.5 bits per weight, 144 bytes per 256."""
+    lib.wq_q4k_bytes.restype = ctypes.c_size_t
+    lib.wq_q4k_bytes.argtypes = [ctypes.c_int64, ctypes.c_int64]
+    assert lib.wq_q4k_bytes(1, 256) == 144
+    assert lib.wq_q4k_bytes(14336, 4096) == 14336 * 4096 * 9 // 16  # 4.5 / 8 bytes per weight
+    assert lib.wq_q4k_bytes(1, 384) == 0 and lib.wq_q4k_bytes(0, 256) == 0
+    assert lib.wq_q4k_bytes(3, 128) == 0
+
+
+def test_superblock_rejections_without_gpu(lib):
+    """Host checks come before any device work: invalid sizes, M and
+    alignment are refused with nothing launched."""
+    vp, i64 = ctypes.c_void_p, ctypes.c_int64
+    lib.wq_q4k_quantize.argtypes = [vp, i64, i64, vp, vp]
+    lib.wq_q4k_quantize.restype = ctypes.c_int
+    lib.wq_q4k_matmul.argtypes = [vp, i64, vp, i64, i64, vp, ctypes.c_int, vp]
+    lib.wq_q4k_matmul.restype = ctypes.c_int
+    buf = ctypes.create_string_buffer(4096 + 32)
+    base = (ctypes.addressof(buf) + 15) // 16 * 16
+    assert lib.wq_q4k_quantize(base, 4, 384, base, None) == 1      # K % 256
+    assert lib.wq_q4k_quantize(None, 4, 256, base, None) == 1      # null W
+    assert lib.wq_q4k_quantize(base + 2, 1, 256, base, None) == 3  # misaligned
+    assert lib.wq_q4k_matmul(base, 9, base, 4, 256, base, 0, None) == 1   # M > 8
+    assert lib.wq_q4k_matmul(base, 1, base, 4, 256, base, 7, None) == 1   # out dtype
+    assert lib.wq_q4k_matmul(base, 1, base + 8, 4, 256, base, 0, None) == 3
+
+
 def test_status_strings(lib):
     lib.wq_status_string.restype = ctypes.c_char_p
     lib.wq_status_string.argtypes = [ctypes.c_int]
