@@ -1,93 +1,92 @@
-"""Paper mode: the pages' own Python-float semantics, for their worked examples.
+"""Paper mode: the pages' affine quantizer in Python floats (binary64).
 
 TEST INFRASTRUCTURE ONLY (see the package docstring).
 
-These functions restate what each page's code computes, in code written for
-this oracle; they keep the pages' precision (Python float = binary64, scales
-not rounded to binary16) and their exact steps:
+Written from the pages' equations, in the pages' precision (binary64,
+scales not rounded to binary16), for their worked examples and the
+information-only error table:
 
-* ``affine_quantize`` -- page 1 ("vLLM 量化与推测解码"), section 1, the
-  per-tensor / per-group executable example: range widened to contain 0,
-  scale = (hi - lo)/(qmax - qmin) or 1.0 for a degenerate range, zero =
-  clamp(round(qmin - lo/scale)), code = clamp(round(v/scale) + zero),
-  reconstruction scale*(code - zero).
-* ``quantize_dequantize_p3`` -- page 3 ("量化：为何加速推理与精度权衡"), section
-  "代码": the same map with the raw min/max (no widening to 0) and no clamp on
-  the zero point; returns the reconstruction and the step.
-* ``quantize_group_symmetric`` / ``dequantize_group_symmetric`` -- page 2
-  ("量化", llminference s08), section "解法": zero point 0, scale = max|w| /
-  (2^(b-1) - 1), codes clipped to [-2^(b-1), 2^(b-1) - 1].
-* ``fused_matmul_kmajor`` -- page 2, section "实现": codes laid out
-  [n_groups, group, out_features] and scales [n_groups, out_features]; the
-  output accumulates one group's dequantized block at a time.
+* ``affine_quantize`` -- page 1 ("vLLM 量化与推测解码"), section 1: the affine
+  map q = clamp(round(x/s) + z, qmin, qmax), x^ = s (q - z) with the
+  min-max calibration s = (x_max - x_min)/(q_max - q_min),
+  z = round(q_min - x_min/s), unsigned b-bit codes (q_min = 0,
+  q_max = 2^b - 1), one (s, z) per group (per tensor when no group size is
+  given).  Where the section's prose leaves a step open, its executable
+  per-tensor / per-group example fixes it: the calibration range is widened
+  to contain real 0, a degenerate range gets s = 1, and z is clamped into
+  [q_min, q_max].
+* ``quantize_dequantize_p3`` -- page 3 ("量化：为何加速推理与精度权衡"),
+  section "直接答案": scale = (h - l)/q_max over the raw range [l, h],
+  z = round(-l/scale) (not clamped), x^ = scale (clamp(round(x/scale) + z,
+  0, q_max) - z); returns x^ and the step (the scale).
+* ``fused_matmul_kmajor`` -- page 2 ("量化", llminference s08), section
+  "实现": the output is the sum over groups of x[:, group g] times group g's
+  dequantized block, with the weights laid out [n_groups, group, out].
 
-``round`` is Python's round(), i.e. round-half-to-even.
+``round`` is half-to-even (``_round``, numpy's rint, the rounding of the
+Python ``round`` that the pages' examples call).
 """
 from __future__ import annotations
 
 import numpy as np
 
+# Round half to even.  A module-level name so that the planted-mistake tests
+# can swap it for a wrong rounding and check that the pins catch it.
+_round = np.rint
+
+
+def _group_starts(n: int, size: int) -> np.ndarray:
+    return np.arange(0, n, size)
+
 
 def affine_quantize(x, bits: int = 8, group_size: int | None = None):
-    """Page 1, section 1.  Returns (codes, reconstruction, [(scale, zero), ...])."""
-    values = [float(v) for v in x]
-    size = len(values) if group_size is None else group_size
-    qmin, qmax = 0, (1 << bits) - 1
-    codes, recon, meta = [], [], []
-    for start in range(0, len(values), size):
-        chunk = values[start:start + size]
-        lo = min(0.0, min(chunk))        # the range always contains real 0
-        hi = max(0.0, max(chunk))
-        scale = 1.0 if hi == lo else (hi - lo) / (qmax - qmin)
-        zero = min(qmax, max(qmin, round(qmin - lo / scale)))
-        for v in chunk:
-            c = min(qmax, max(qmin, round(v / scale) + zero))
-            codes.append(c)
-            recon.append(scale * (c - zero))
-        meta.append((scale, zero))
-    return codes, recon, meta
+    """Page 1, section 1: groupwise affine quantization of a 1-D sequence.
+
+    Returns (codes, reconstruction, [(scale, zero) per group]) as Python
+    lists; the last group may be shorter than ``group_size``."""
+    v = np.asarray([float(e) for e in x], dtype=np.float64)
+    n = v.size
+    size = n if group_size is None else int(group_size)
+    q_min, q_max = 0.0, float((1 << bits) - 1)
+    starts = _group_starts(n, size)
+    # calibration range of each group, widened to contain real 0
+    x_min = np.minimum(np.minimum.reduceat(v, starts), 0.0)
+    x_max = np.maximum(np.maximum.reduceat(v, starts), 0.0)
+    degenerate = x_max == x_min
+    s = np.where(degenerate, 1.0, (x_max - x_min) / np.where(degenerate, 1.0, q_max - q_min))
+    z = np.clip(_round(q_min - x_min / s), q_min, q_max)
+    g = np.arange(n) // size                      # group of each element
+    q = np.clip(_round(v / s[g]) + z[g], q_min, q_max)
+    x_hat = s[g] * (q - z[g])
+    codes = [int(c) for c in q]
+    meta = [(float(a), int(b)) for a, b in zip(s, z)]
+    return codes, [float(e) for e in x_hat], meta
 
 
 def quantize_dequantize_p3(xs, bits: int):
-    """Page 3, "代码".  Returns (reconstruction, scale)."""
-    qmax = (1 << bits) - 1
-    lo, hi = min(xs), max(xs)
-    scale = (hi - lo) / qmax
-    zero = round(-lo / scale)
-    recon = []
-    for v in xs:
-        c = min(qmax, max(0, round(v / scale) + zero))
-        recon.append(scale * (c - zero))
-    return recon, scale
-
-
-def quantize_group_symmetric(w, bits: int = 4):
-    """Page 2, "解法" (symmetric, one scale per group).  ``w`` is a 1-D array
-    of one group.  Returns (int codes, scale as binary16)."""
-    w = np.asarray(w, dtype=np.float64)
-    qmax = (1 << (bits - 1)) - 1
-    scale = float(np.abs(w).max()) / qmax
-    q = np.clip(np.round(w / scale), -qmax - 1, qmax).astype(np.int64)
-    return q, np.float16(scale)
-
-
-def dequantize_group_symmetric(q, scale) -> np.ndarray:
-    """Page 2, "解法": q * scale."""
-    return np.asarray(q, dtype=np.float64) * float(scale)
+    """Page 3, "直接答案": one scale over the raw range; returns
+    (reconstruction as a list, scale)."""
+    v = np.asarray([float(e) for e in xs], dtype=np.float64)
+    q_max = float((1 << bits) - 1)
+    l, h = float(v.min()), float(v.max())
+    scale = (h - l) / q_max
+    z = _round(-l / scale)
+    q = np.clip(_round(v / scale) + z, 0.0, q_max)
+    return [float(e) for e in scale * (q - z)], scale
 
 
 def fused_matmul_kmajor(x, q_kmajor, scales_kmajor, group: int) -> np.ndarray:
-    """Page 2, "实现": out += x[:, group g] @ (q[g] * scales[g]) for each g.
+    """Page 2, "实现": Y = sum over groups g of x[:, g-th group of K] times
+    (q[g] * scales[g]).
 
-    ``x`` is [M, K] float64, ``q_kmajor`` is [n_groups, group, out_features]
+    ``x`` is [M, K], ``q_kmajor`` is [n_groups, group, out_features]
     integer-valued (here already q - z), ``scales_kmajor`` is [n_groups,
-    out_features].  Everything in float64, one group block at a time.
-    """
+    out_features]; everything in binary64."""
     n_groups, gsize, out_f = q_kmajor.shape
     assert gsize == group
     x = np.asarray(x, dtype=np.float64)
-    out = np.zeros((x.shape[0], out_f), dtype=np.float64)
-    for g in range(n_groups):
-        block = q_kmajor[g].astype(np.float64) * scales_kmajor[g].astype(np.float64)
-        out += x[:, g * group:(g + 1) * group] @ block
-    return out
+    blocks = q_kmajor.astype(np.float64) * scales_kmajor.astype(np.float64)[:, None, :]
+    x_groups = x.reshape(x.shape[0], n_groups, group)
+    # one group's partial product per g, then their sum
+    partial = np.einsum("mgk,gko->gmo", x_groups, blocks)
+    return partial.sum(axis=0)

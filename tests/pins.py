@@ -97,7 +97,7 @@ def check_half_round_up(orc):
 
 # ------------------------------------------------------- worked examples
 
-def check_p1_example_paper_mode():
+def check_p1_example_paper_mode(paper=paper):
     """Page 1 section 1 example in the page's own float semantics.
 
     Per tensor (group = 8): lo = -8, hi = 7.3, s = 15.3/15 = 1.02,
@@ -151,21 +151,35 @@ def check_p1_example_storage_mode(orc):
     assert codes.tolist() == [[0 | 14 << 4, 14 | 15 << 4, 14 | 15 << 4, 15 | 15 << 4]]
 
 
-def check_p3_example(orc, golden):
+def check_p3_example_paper_mode(golden, paper=paper):
     """Page 3 "代码": INT4 on [-0.9, -0.2, 0.1, 0.5, 3.0] prints step 0.26 and
     bound 0.13.  By hand: s = 3.9/15 = 0.26, z = round(0.9/0.26 = 3.46) = 3,
     round(v/s) = [-3, -1, 0, 2, 12] -> codes [0, 2, 3, 5, 15],
-    x^ = [-0.78, -0.26, 0, 0.52, 3.12], max error 0.12 <= 0.13.
-    Storage mode: lo = -0.89990234375 (binary16 of -0.9), (3 + 0.8999)/15 =
-    0.2599935; spacing 2^-12 -> 1064.93 ulps -> 1065 * 2^-12 = 0.260009765625;
-    same codes."""
+    x^ = [-0.78, -0.26, 0, 0.52, 3.12], max error 0.12 <= 0.13.  Page 1's
+    quantizer (range widened to contain 0: the example already straddles 0)
+    gives the same codes and zero."""
     xs = [-0.9, -0.2, 0.1, 0.5, 3.0]
     recon, step = paper.quantize_dequantize_p3(xs, 4)
     assert f"{step:.2f}" == golden["printed_step"]
     assert f"{step / 2:.2f}" == golden["printed_bound"]
     assert max(abs(a - b) for a, b in zip(xs, recon)) <= step / 2
-    codes_p1, _, meta = paper.affine_quantize(xs, bits=4)
+    want = [-0.78, -0.26, 0.0, 0.52, 3.12]
+    assert all(abs(a - b) < 1e-12 for a, b in zip(recon, want)), recon
+    codes_p1, recon_p1, meta = paper.affine_quantize(xs, bits=4)
     assert codes_p1 == [0, 2, 3, 5, 15] and meta[0][1] == 3
+    assert all(abs(a - b) < 1e-12 for a, b in zip(recon_p1, want)), recon_p1
+    # the clamp of the page's code at work: on [-3.5, 11.5] the scale is 1,
+    # z = round(3.5) = 4 and round(11.5) + 4 = 16 -> clamped to 15, x^ = 11
+    recon, step = paper.quantize_dequantize_p3([-3.5, 11.5], 4)
+    assert step == 1.0 and recon == [-4.0, 11.0]
+
+
+def check_p3_example(orc, golden):
+    """Page 3 "代码" example through the storage-mode oracle: lo =
+    -0.89990234375 (binary16 of -0.9), (3 + 0.8999)/15 = 0.2599935; spacing
+    2^-12 -> 1064.93 ulps -> 1065 * 2^-12 = 0.260009765625; codes
+    [0, 2, 3, 5, 15] as worked by hand in check_p3_example_paper_mode."""
+    xs = [-0.9, -0.2, 0.1, 0.5, 3.0]
     W = to_half_bits([xs + [0.0]])                # pad to an even length for packing
     q, _, s, z = orc.quantize(W[:, :5].copy(), 4, 5, False, pack=False)
     assert half_values(s).ravel().tolist() == [0.260009765625]
@@ -173,6 +187,53 @@ def check_p3_example(orc, golden):
     assert q.tolist() == [[0, 2, 3, 5, 15]]
     what = 0.260009765625 * (np.array([0, 2, 3, 5, 15]) - 3)
     assert np.max(np.abs(half_values(W[0, :5]) - what)) <= 0.13
+    assert f"{0.260009765625:.2f}" == golden["printed_step"]
+
+
+def check_paper_degenerate_and_zero(paper=paper):
+    """Page 1 section 1's example code: a degenerate range gets scale 1.0 and
+    zero 0, so an all-zero group comes back as zeros; the widened range keeps
+    real 0 exact in every group (page 3 "深入原理")."""
+    codes, recon, meta = paper.affine_quantize([0.0] * 4 + [0.5, 1.0, 0.0, 2.0], bits=4,
+                                               group_size=4)
+    assert meta[0] == (1.0, 0) and codes[:4] == [0, 0, 0, 0] and recon[:4] == [0.0] * 4
+    assert meta[1][1] == 0 and abs(meta[1][0] - 2.0 / 15) < 1e-15   # lo widened to 0
+    assert recon[6] == 0.0
+    codes, recon, _ = paper.affine_quantize([-3.0, 0.0, 1.0, 0.0, 5.0, -0.25], bits=3,
+                                            group_size=3)
+    assert recon[1] == 0.0 and recon[3] == 0.0
+
+
+def check_paper_ties_to_even(paper=paper):
+    """A 4-bit group on [0, 15/64] has s = 2^-6 and z = 0 exactly in binary64;
+    the weights (j + 1/2)/64 sit exactly between codes j and j + 1 and go to
+    the even one (Python's round, which the pages' code calls)."""
+    vals = [0.0, 15 / 64] + [(j + 0.5) / 64 for j in range(14)]
+    codes, _, meta = paper.affine_quantize(vals, bits=4)
+    assert meta == [(1 / 64, 0)]
+    assert codes == [0, 15] + [j if j % 2 == 0 else j + 1 for j in range(14)]
+    neg = [-v for v in vals]                     # z = 15 on the mirrored group
+    codes, _, meta = paper.affine_quantize(neg, bits=4)
+    assert meta == [(1 / 64, 15)]
+    assert codes == [15, 0] + [15 - (j if j % 2 == 0 else j + 1) for j in range(14)]
+
+
+def check_paper_nearest_and_bound(paper=paper, seed=11):
+    """Page 1 section 1's quantizer in binary64 on random groups with an
+    outlier: every code is the nearest of the 2^b grid points s (c - z)
+    (brute force), and |x - x^| <= s/2 (page 3 "直接答案") up to binary64
+    rounding of x/s."""
+    rng = np.random.default_rng(seed)
+    for bits in (2, 3, 4, 8):
+        x = rng.normal(0.0, 0.02, 96)
+        x[17] *= 40.0
+        codes, recon, meta = paper.affine_quantize(x, bits=bits, group_size=32)
+        for i, v in enumerate(x):
+            s, z = meta[i // 32]
+            grid = [s * (c - z) for c in range(1 << bits)]
+            best = min(abs(v - gv) for gv in grid)
+            assert abs(v - s * (codes[i] - z)) <= best + 1e-15, (bits, i)
+            assert abs(v - recon[i]) <= s / 2 * (1 + 1e-12), (bits, i)
 
 
 def check_payload(orc, golden):
@@ -391,7 +452,7 @@ def check_matmul_exact_sum(orc, bits, group, symmetric, W, seed=7):
             assert abs(Fraction(Y[m, n]) - exact) <= Fraction(Yabs[m, n]) * Fraction(1, 10**12)
 
 
-def check_matmul_kmajor(orc, bits, group, symmetric, W, seed=8):
+def check_matmul_kmajor(orc, bits, group, symmetric, W, seed=8, paper=paper):
     """Page 2 "实现": accumulating x[:, group g] @ (q[g] * scale[g]) group by
     group over a [n_groups, group, out] layout gives the same Y (codes here
     already have the zero point subtracted)."""

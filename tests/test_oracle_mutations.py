@@ -89,3 +89,70 @@ def test_planted_mistake_is_caught(tmp_path, name, old, new):
     # build reuse its inode, and the dynamic loader would hand back this
     # library instead of the new one
     assert caught, f"no pin caught the planted mistake '{name}'"
+
+
+# ------------------------------------------------------------ paper mode
+# The same for the binary64 paper-mode module (oracle/paper.py): each
+# mistake is planted in a copy of its source, loaded as a separate module.
+
+PAPER_SRC = open(os.path.join(os.path.dirname(oracle.SOURCE), "paper.py")).read()
+
+PAPER_MUTANTS = [
+    ("paper: rounding truncates", "_round = np.rint", "_round = np.trunc"),
+    ("paper: rounding half away from zero", "_round = np.rint",
+     "_round = lambda t: np.sign(t) * np.floor(np.abs(t) + 0.5)"),
+    ("paper: range not widened to 0",
+     "x_min = np.minimum(np.minimum.reduceat(v, starts), 0.0)",
+     "x_min = np.minimum.reduceat(v, starts)"),
+    ("paper: zero point with the wrong sign",
+     "z = np.clip(_round(q_min - x_min / s), q_min, q_max)",
+     "z = np.clip(_round(q_min + x_min / s), q_min, q_max)"),
+    ("paper: reconstruction drops the zero point",
+     "x_hat = s[g] * (q - z[g])", "x_hat = s[g] * q"),
+    ("paper: degenerate scale not 1", "s = np.where(degenerate, 1.0,", "s = np.where(degenerate, 0.5,"),
+    ("paper: group size ignored",
+     "size = n if group_size is None else int(group_size)", "size = n"),
+    ("paper: page 3 step over 2^b levels",
+     "scale = (h - l) / q_max", "scale = (h - l) / (q_max + 1.0)"),
+    ("paper: page 3 codes not clamped",
+     "q = np.clip(_round(v / scale) + z, 0.0, q_max)", "q = _round(v / scale) + z"),
+    ("paper: K-major product drops the scale",
+     "blocks = q_kmajor.astype(np.float64) * scales_kmajor.astype(np.float64)[:, None, :]",
+     "blocks = q_kmajor.astype(np.float64) + 0.0 * scales_kmajor.astype(np.float64)[:, None, :]"),
+    ("paper: K-major groups taken strided",
+     "x_groups = x.reshape(x.shape[0], n_groups, group)",
+     "x_groups = x.reshape(x.shape[0], group, n_groups).transpose(0, 2, 1)"),
+]
+
+
+def _paper_checks(mod):
+    orc = oracle.get()
+    golden = {"printed_step": "0.26", "printed_bound": "0.13"}
+    return [
+        ("p1 paper example", lambda: pins.check_p1_example_paper_mode(mod)),
+        ("p3 paper example", lambda: pins.check_p3_example_paper_mode(golden, mod)),
+        ("paper degenerate / zero", lambda: pins.check_paper_degenerate_and_zero(mod)),
+        ("paper ties to even", lambda: pins.check_paper_ties_to_even(mod)),
+        ("paper nearest / bound", lambda: pins.check_paper_nearest_and_bound(mod)),
+        ("K-major matmul", lambda: pins.check_matmul_kmajor(
+            orc, 4, 32, False, _w(6, 128, 9), paper=mod)),
+    ]
+
+
+@pytest.mark.parametrize("name,old,new", PAPER_MUTANTS, ids=[m[0] for m in PAPER_MUTANTS])
+def test_planted_paper_mistake_is_caught(tmp_path, name, old, new):
+    import importlib.util
+    assert PAPER_SRC.count(old) == 1, f"snippet for '{name}' not found exactly once"
+    path = tmp_path / "paper_planted.py"
+    path.write_text(PAPER_SRC.replace(old, new))
+    spec = importlib.util.spec_from_file_location("paper_planted", str(path))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    caught = []
+    for check_name, fn in _paper_checks(mod):
+        try:
+            fn()
+        except (AssertionError, ValueError, IndexError):
+            caught.append(check_name)
+            break
+    assert caught, f"no pin caught the planted mistake '{name}'"

@@ -42,6 +42,22 @@ def test_p3_example(orc):
     pins.check_p3_example(orc, GOLDEN["p3_example"])
 
 
+def test_p3_example_paper_mode():
+    pins.check_p3_example_paper_mode(GOLDEN["p3_example"])
+
+
+def test_paper_degenerate_and_zero():
+    pins.check_paper_degenerate_and_zero()
+
+
+def test_paper_ties_to_even():
+    pins.check_paper_ties_to_even()
+
+
+def test_paper_nearest_and_bound():
+    pins.check_paper_nearest_and_bound()
+
+
 def test_payload_bytes(orc):
     pins.check_payload(orc, GOLDEN)
 
