@@ -41,17 +41,27 @@ BITS, GROUP, SYM = 4, 128, False
 WORKLOAD = ("decode GEMV, Llama-8B gate/up layer: M=1, K=4096, N=14336, INT4 asymmetric "
             "group 128, fp16 scale+zero, bf16 X, fp32 Y")
 FALLBACK_HBM_GBS = 6650.0
+GRAPH_MAX_LAUNCHES = 4096      # larger step counts replay graphs of one pool cycle
+SLEEP_CYCLES = 2_000_000       # ~1 ms of device time ahead of the start event
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "gemv_w4a16_m1_k4096_n14336.json")
 CSRC = os.path.join(ROOT, "w4a16_decode_matmul_b200", "csrc")
 # What decides the timed kernel: its device code, the host plan and launch of
 # it, and the matmul entry point that chooses it.
-KERNEL_SOURCES = [os.path.join(CSRC, f) for f in ("gemv_ld.cuh", "unpack.cuh", "common.cuh")]
+KERNEL_SOURCES = [os.path.join(CSRC, f)
+                  for f in ("gemv_ld.cuh", "unpack.cuh", "common.cuh", "k_ld.cu")]
 KERNEL_HOST_SECTIONS = [
-    ("// --------------------------------------------------- direct-load kernel",
-     "// ------------------------------------------------------- balanced kernel"),
     ("wq_status wq_matmul(const void* X, int64_t M,",
      "// ------------------------------------------------------ no-allocation entry"),
 ]
+# Page 2 ("量化", llminference s08, section 换来了什么): its bandwidth-model
+# estimate for an 8B model on an H100 (~3.35 TB/s), quoted as context only.
+PAGE2_H100_CONTEXT = {
+    "kind": "context from the pages (another GPU, a bytes / bandwidth model), not a target",
+    "source": "page 2 '量化' (llminference s08), section 换来了什么: 8B model on an H100",
+    "fp16_ms_per_token": 4.78, "int4_group32_ms_per_token": 1.25,
+    "note": ("the 1.25 ms uses 4.19 GiB as if it were GB; with 8e9 x 4.5 / 8 = 4.5e9 bytes "
+             "the same model gives 1.34 ms"),
+}
 
 
 def algorithmic_bytes(m: int = M, n: int = N, k: int = K, bits: int = BITS,
@@ -63,8 +73,8 @@ def algorithmic_bytes(m: int = M, n: int = N, k: int = K, bits: int = BITS,
 
 
 def kernel_source_hash() -> str:
-    """Hash of the sources that decide the timed kernel (device headers, and
-    the sections of wq.cu that plan, choose and launch it)."""
+    """Hash of the sources that decide the timed kernel (device headers, its
+    plan and launch in k_ld.cu, and the kernel choice in wq.cu)."""
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
         h.update(open(f, "rb").read())
@@ -173,17 +183,24 @@ def oracle_threads() -> int:
     return len(os.sched_getaffinity(0))
 
 
-def time_oracle(target_s: float, seed_w: int = 0, seed_x: int = 1):
+_ORACLE_INPUTS = {}
+
+
+def time_oracle(target_s: float, seed_w: int = 0, seed_x: int = 1, threads: int | None = None):
     """Time the oracle's matmul (decode from codes + float64 dot products) on
-    the same layer for about target_s seconds.  Returns (GB/s, steps, s)."""
-    os.environ.setdefault("OMP_NUM_THREADS", str(oracle_threads()))
+    the same layer for about target_s seconds, with `threads` OpenMP threads
+    (all affinity cores by default).  Returns (GB/s, steps, s)."""
     import oracle
     import synth
-    W = synth.weight(N, K, seed=seed_w)
-    X = synth.activation(M, K, seed=seed_x)
     orc = oracle.get()
-    _, codes, scales, zeros = orc.quantize(synth.half_bits(W), BITS, GROUP, SYM)
-    xb = synth.bf16_bits(X)
+    key = (seed_w, seed_x)
+    if key not in _ORACLE_INPUTS:
+        W = synth.weight(N, K, seed=seed_w)
+        X = synth.activation(M, K, seed=seed_x)
+        _, codes, scales, zeros = orc.quantize(synth.half_bits(W), BITS, GROUP, SYM)
+        _ORACLE_INPUTS[key] = (codes, scales, zeros, synth.bf16_bits(X))
+    codes, scales, zeros, xb = _ORACLE_INPUTS[key]
+    orc.set_threads(threads or oracle_threads())
     steps, t0 = 0, time.perf_counter()
     while True:
         orc.matmul(xb, codes, scales, zeros, N, K, BITS, GROUP, SYM)
@@ -204,7 +221,7 @@ def run_reference(args):
         time_oracle(0.0)
     target = max(5.0, min(30.0, 0.05 * args.steps))
     gbs, steps, el = time_oracle(target)
-    cores = int(os.environ.get("OMP_NUM_THREADS", oracle_threads()))
+    cores = oracle_threads()
     sample = (f"oracle matmul over the full {K}x{N} layer at M=1, {steps} steps in "
               f"{el:.1f} s (bounded sample of the benchmark's step count)")
     line = {
@@ -265,13 +282,22 @@ def run_wq(args):
         return g
 
     steps = args.steps
-    full, rest = divmod(steps, pool_n)
-    g_full = capture(pool_n)
-    g_rest = capture(rest) if rest else None
-
+    warm = max(args.warmup, 3)
+    # The timed launches are replayed from CUDA graphs: one graph of exactly
+    # `steps` launches when that is small, else a graph of one pool cycle
+    # replayed `full` times plus one of the `rest`.  Every graph is replayed
+    # before the timed region, so that no first-replay cost is timed.
+    if steps <= GRAPH_MAX_LAUNCHES:
+        graphs = [(capture(steps), 1)]
+    else:
+        full, rest = divmod(steps, pool_n)
+        graphs = [(capture(pool_n), full)] + ([(capture(rest), 1)] if rest else [])
+    g_cycle = capture(pool_n)            # for the per-replay distribution
     with torch.cuda.stream(stream):
-        for _ in range(max(1, -(-max(args.warmup, 3) // pool_n))):
-            g_full.replay()
+        for g, _ in graphs:
+            g.replay()
+        for _ in range(max(1, -(-warm // pool_n))):
+            g_cycle.replay()
     stream.synchronize()
 
     start = torch.cuda.Event(enable_timing=True)
@@ -281,11 +307,13 @@ def run_wq(args):
     torch.cuda.synchronize(dev)
     with ClockSampler(f"GPU-{torch.cuda.get_device_properties(dev).uuid}") as clocks:
         with torch.cuda.stream(stream):
+            # a short device-side wait ahead of the start event, so that the
+            # host has queued every replay before the timed region begins
+            torch.cuda._sleep(SLEEP_CYCLES)
             start.record(stream)
-            for _ in range(full):
-                g_full.replay()
-            if g_rest is not None:
-                g_rest.replay()
+            for g, n in graphs:
+                for _ in range(n):
+                    g.replay()
             end.record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
@@ -308,7 +336,7 @@ def run_wq(args):
 
     # comparison points on the same GPU (not part of the timed region)
     extra = compare_points(wq, torch, dev, stream, pool, X, pool_n)
-    extra["per_graph_distribution"] = graph_distribution(torch, dev, stream, g_full, pool_n)
+    extra["per_graph_distribution"] = graph_distribution(torch, dev, stream, g_cycle, pool_n)
     extra["warm_l2"] = warm_l2_point(wq, torch, dev, stream, pool[0], X)
     extra["stream_read_ceiling"] = stream_ceiling(wq, torch, dev, stream, pool, pool_n)
     extra["stream_read_ceiling"]["fused_frac_of_ceiling"] = round(
@@ -318,8 +346,7 @@ def run_wq(args):
     e2e = measure_e2e(wq, torch, dev, pool, pool_n, args)
 
     # the prefill row (tensor cores), outside the timed region
-    del pool, g_full, g_rest
-    g_full = g_rest = None
+    del pool, graphs, g_cycle
     prefill = prefill_points(wq, torch, dev)
     # the quantize rows: the benchmark layer, then every matrix of the model
     quant = quantize_points(wq, torch, dev, stream)
@@ -336,7 +363,10 @@ def run_wq(args):
                    "l2": (f"rotating pool of {pool_n} weight copies "
                           f"({pool_n * layer_bytes / 1e6:.0f} MB, "
                           f"{pool_n * layer_bytes / l2:.1f}x the {l2 / 1e6:.0f} MB L2)"),
-                   "timing": f"CUDA graphs of {pool_n} launches, CUDA events on the launch stream",
+                   "timing": ("CUDA graphs (" + ("one graph of all steps" if steps <= GRAPH_MAX_LAUNCHES
+                                                 else f"{pool_n}-launch cycles") +
+                              ", each replayed once before timing), CUDA events on the launch "
+                              "stream"),
                    "launch": "programmatic dependent launch (static weights)"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
@@ -352,19 +382,22 @@ def run_wq(args):
         "quantize_layer": quant,
         "quantize_whole_model": model_quant,
         "q4k_gemv": q4k,
+        "page2_h100_bandwidth_model": PAGE2_H100_CONTEXT,
     }
     if world == 1:
-        gbs, st, el = time_oracle(10.0)
+        cores = oracle_threads()
+        gbs, st, el = time_oracle(8.0, threads=cores)
+        gbs1, st1, el1 = time_oracle(6.0, threads=1)
         line["cpu_baseline"] = {
-            "value": round(gbs, 4), "unit": "GB/s",
-            "cores": int(os.environ.get("OMP_NUM_THREADS", oracle_threads())),
-            "kind": "oracle",
-            "sample": f"oracle matmul over the full {K}x{N} layer at M=1, {st} steps in {el:.1f} s"}
+            "value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": (f"oracle matmul over the full {K}x{N} layer at M=1, {st} steps in "
+                       f"{el:.1f} s on {cores} threads"),
+            "single_thread": {"value": round(gbs1, 4), "unit": "GB/s", "cores": 1,
+                              "sample": f"{st1} steps in {el1:.1f} s"}}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
-        del g_full, g_rest
         dist.destroy_process_group()
     return 0
 
@@ -647,54 +680,144 @@ def measured_bf16_tflops():
     return 1590.0
 
 
+def _cudart():
+    """ctypes handle on the CUDA runtime that torch loads (for plain
+    cudaMemcpyAsync calls in the end-to-end loop), or None."""
+    import ctypes
+    import glob
+    import nvidia
+    for d in nvidia.__path__:
+        for path in sorted(glob.glob(os.path.join(d, "cuda_runtime", "lib", "libcudart.so*"))):
+            try:
+                rt = ctypes.CDLL(path)
+            except OSError:
+                continue
+            rt.cudaMemcpyAsync.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                           ctypes.c_int, ctypes.c_void_p]
+            rt.cudaMemcpyAsync.restype = ctypes.c_int
+            rt.cudaStreamSynchronize.argtypes = [ctypes.c_void_p]
+            rt.cudaStreamSynchronize.restype = ctypes.c_int
+            return rt
+    return None
+
+
 def measure_e2e(wq, torch, dev, pool, pool_n, args):
-    """Public API with host buffers: pinned X copied in, Y read back, every
-    step, inside the timed region."""
+    """End to end through the C ABI with host buffers: every step copies X
+    from pinned host memory to the device (cudaMemcpyAsync), calls
+    wq_matmul, copies Y back to pinned host memory and waits for it (the
+    host reads Y), all inside the timed region (wall clock, max with the
+    device events)."""
+    import ctypes
     import synth
+    lib = wq.lib
+    rt = _cudart()
     Xh = synth.activation(M, K, seed=1).pin_memory()
     Yh = torch.empty(M, N, dtype=torch.float32).pin_memory()
-    steps = max(50, min(2000, args.steps // 100))
-    for i in range(5):
-        wq.matmul(Xh, pool[i % pool_n], out=Yh)
-        torch.cuda.current_stream(dev).synchronize()
-    t0 = time.perf_counter()
-    s = torch.cuda.Event(enable_timing=True)
-    e = torch.cuda.Event(enable_timing=True)
-    s.record()
-    for i in range(steps):
-        wq.matmul(Xh, pool[i % pool_n], out=Yh)
-        torch.cuda.current_stream(dev).synchronize()     # the host reads Y
-    e.record()
-    torch.cuda.synchronize(dev)
-    wall = time.perf_counter() - t0
+    Xd = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    Yd = torch.empty(M, N, dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(dev)
+    h = ctypes.c_void_p(stream.cuda_stream)
+    ws = wq.workspace(dev, stream.cuda_stream)
+    vp = ctypes.c_void_p
+    x_bytes, y_bytes = M * K * 2, M * N * 4
+    calls = []
+    for q in pool:
+        calls.append((vp(Xd.data_ptr()), M, vp(q.codes.data_ptr()), vp(q.scales.data_ptr()),
+                      None if q.zeros is None else vp(q.zeros.data_ptr()), N, K, BITS, GROUP,
+                      int(SYM), vp(Yd.data_ptr()), wq.WQ_OUT_F32, vp(ws.data_ptr()), ws.numel(),
+                      0, h))
+
+    def step(i):
+        if rt is not None:
+            rt.cudaMemcpyAsync(vp(Xd.data_ptr()), vp(Xh.data_ptr()), x_bytes, 1, h)
+        else:
+            with torch.cuda.stream(stream):
+                Xd.copy_(Xh, non_blocking=True)
+        st = lib.wq_matmul(*calls[i % pool_n])
+        if st != 0:
+            raise wq.WQError(st, "wq_matmul")
+        if rt is not None:
+            rt.cudaMemcpyAsync(vp(Yh.data_ptr()), vp(Yd.data_ptr()), y_bytes, 2, h)
+            rt.cudaStreamSynchronize(h)
+        else:
+            with torch.cuda.stream(stream):
+                Yh.copy_(Yd, non_blocking=True)
+            stream.synchronize()
+
+    steps = max(200, min(5000, args.steps))
+    with torch.cuda.device(dev):
+        for i in range(20):
+            step(i)
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        t0 = time.perf_counter()
+        s.record(stream)
+        for i in range(steps):
+            step(i)
+        e.record(stream)
+        torch.cuda.synchronize(dev)
+        wall = time.perf_counter() - t0
     ms = reduce_max(max(s.elapsed_time(e), wall * 1e3), dev)
     _, world, _ = dist_env()
     return {"value": round(whole_job_gbs(algorithmic_bytes(), steps, world, ms), 3),
-            "unit": "GB/s", "h2d_bytes_per_step": M * K * 2,
-            "d2h_bytes_per_step": M * N * 4, "steps": steps,
-            "us_per_step": round(ms / steps * 1e3, 3)}
+            "unit": "GB/s", "h2d_bytes_per_step": x_bytes, "d2h_bytes_per_step": y_bytes,
+            "steps": steps, "us_per_step": round(ms / steps * 1e3, 3),
+            "how": ("C ABI wq_matmul per step between cudaMemcpyAsync of X (pinned host -> "
+                    "device) and of Y (device -> pinned host) and a stream synchronize")}
 
 
-def ncu_case():
-    """A small, self-contained launch sequence for ncu captures: one
-    quantize of the benchmark layer, 8 fused decode matmuls (M=1) on it,
-    then 2 prefill matmuls (M=2048) on it."""
+def ncu_case(which: str = "decode"):
+    """Small, self-contained launch sequences for ncu captures (no timing):
+
+    decode   -- quantize the benchmark layer, 8 fused decode matmuls (M=1),
+                then 2 prefill matmuls (M=2048) on it;
+    traffic  -- the same layer through the three paths page 2 "实现" compares,
+                3 launches each: the fused matmul; the unfused path
+                (dequantize to bf16, then a cuBLAS bf16 GEMV); the dense bf16
+                GEMV on a bf16 weight of the same shape;
+    prefill  -- 2 prefill matmuls at M=2048;
+    quantize -- 3 quantize launches over 3 different 117 MB layers;
+    q4k      -- superblock quantize, then 4 superblock decode matmuls."""
     import torch
     import synth
     import w4a16_decode_matmul_b200 as wq
     dev = torch.device("cuda", 0)
-    qw = wq.quantize(synth.weight(N, K, seed=0).to(dev), bits=BITS, group=GROUP, symmetric=SYM)
+    torch.cuda.set_device(dev)
+    W = synth.weight(N, K, seed=0).to(dev)
     X = synth.activation(M, K, seed=1).to(dev)
     Y = torch.empty(M, N, dtype=torch.float32, device=dev)
-    for _ in range(8):
-        wq.matmul(X, qw, out=Y)
-    Xp = synth.activation(2048, K, seed=2).to(dev)
-    Yp = torch.empty(2048, N, dtype=torch.float32, device=dev)
-    for _ in range(2):
-        wq.matmul(Xp, qw, out=Yp)
+    if which in ("decode", "traffic", "prefill"):
+        qw = wq.quantize(W, bits=BITS, group=GROUP, symmetric=SYM)
+    if which == "decode":
+        for _ in range(8):
+            wq.matmul(X, qw, out=Y)
+    if which in ("decode", "prefill"):
+        Xp = synth.activation(2048, K, seed=2).to(dev)
+        Yp = torch.empty(2048, N, dtype=torch.float32, device=dev)
+        for _ in range(2):
+            wq.matmul(Xp, qw, out=Yp)
+    if which == "traffic":
+        Wt = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
+        Wd = W.to(torch.bfloat16)
+        Yb = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            wq.matmul(X, qw, out=Y)
+        for _ in range(3):
+            wq.dequantize(qw, out=Wt)
+            torch.matmul(X, Wt.T, out=Yb)
+        for _ in range(3):
+            torch.matmul(X, Wd.T, out=Yb)
+    if which == "quantize":
+        Ws = [synth.weight(N, K, seed=10 + i, device=dev) for i in range(3)]
+        for Wi in Ws:
+            wq.quantize(Wi, bits=BITS, group=GROUP, symmetric=SYM)
+    if which == "q4k":
+        blocks = wq.q4k_quantize(W)
+        for _ in range(4):
+            wq.q4k_matmul(X, blocks, N, K, out=Y)
     torch.cuda.synchronize(dev)
     assert wq.get_device_error(dev) == 0
-    print("ncu case ok")
+    print(f"ncu case {which} ok")
     return 0
 
 
@@ -704,11 +827,12 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200000)
     ap.add_argument("--warmup", type=int, default=2000)
     ap.add_argument("--impl", choices=["wq", "reference"], default="wq")
-    ap.add_argument("--ncu-case", action="store_true",
-                    help="no timing: quantize the layer, run 8 decode and 2 prefill matmuls, for ncu")
+    ap.add_argument("--ncu-case", nargs="?", const="decode", default=None,
+                    choices=["decode", "traffic", "prefill", "quantize", "q4k"],
+                    help="no timing: a short launch sequence for ncu captures (see ncu_case)")
     args = ap.parse_args(argv)
     if args.ncu_case:
-        return ncu_case()
+        return ncu_case(args.ncu_case)
     if args.impl == "reference":
         return run_reference(args)
     return run_wq(args)

@@ -132,9 +132,17 @@ size_t wq_matmul_workspace_bytes(void);
 /* Y [M][N] = X [M][K] * What^T, weights formed on chip from codes, scales
  * and zeros and never written to memory.  out_dtype is WQ_OUT_F32 or
  * WQ_OUT_BF16 (round-to-nearest-even from the binary32 accumulator).
- * M <= 32 runs the small-batch decode kernels (codes streamed once from HBM,
- * tensor-core products of integer-valued bfloat16 codes, binary32 group
- * scaling); M > 32 returns WQ_ERR_UNSUPPORTED in this build.
+ *
+ * M <= 32 runs the small-batch decode kernels: codes streamed once from
+ * HBM, tensor-core products of integer-valued 16-bit codes, binary32 group
+ * scaling.  Every supported format is accepted.
+ *
+ * M > 32 runs the prefill kernel: the exact integers q - z on the tcgen05
+ * tensor cores with binary32 accumulators in tensor memory, one per group,
+ * scaled by s in binary32 ("量化" (llminference s08) section 实现: large
+ * batches are bound by the multiply).  Its scope in this build: group 64 or
+ * 128, K a multiple of 64 with K/group a multiple of 8 and at most 256;
+ * other formats at M > 32 return WQ_ERR_UNSUPPORTED.
  *
  * workspace / workspace_bytes: NULL and 0, or a buffer of at least
  * wq_matmul_workspace_bytes() bytes as described there.  With it, every SM
@@ -152,17 +160,24 @@ wq_status wq_matmul(const void *X, int64_t M, const void *codes, const void *sca
                     int symmetric, void *Y, int out_dtype, void *workspace,
                     size_t workspace_bytes, unsigned int flags, wq_stream_t stream);
 
-/* As wq_matmul, without a workspace argument and without allocating: the
- * workspace is a fixed block of device memory inside the library
- * (wq_matmul_noalloc_scratch_bytes() bytes, zero at load, left zero by every
- * completed call), found with cudaGetSymbolAddress on the first call on
- * each device and cleared then.  The pages have no counterpart of this entry
- * point; it exists for callers that must not allocate (for example inside a
- * captured CUDA graph).
- *   - Make the first call on a device before any stream capture (the look-up
- *     and the clearing are synchronous).
+/* As wq_matmul, without a workspace argument and without allocating:
+ * the workspace is a fixed block of device memory inside the library
+ * (wq_matmul_noalloc_scratch_bytes() bytes: flags and partial sums for up to
+ * 1,024 CTAs), zero at load and left zero by every completed call.  The
+ * pages have no counterpart of this entry point.  It is for callers that
+ * cannot call cudaMalloc: code that runs where the allocator must not be
+ * entered (a host callback, a real-time or signal-safe path, a custom
+ * allocator that owns all device memory), or that must not grow its memory
+ * after start-up.
+ *   - The first call on a device looks up the block's address with
+ *     cudaGetSymbolAddress (with that device current) and clears the block,
+ *     synchronously (cudaMemset, then cudaDeviceSynchronize): make that
+ *     first call before any stream capture.
  *   - All calls on a device share the block: calls whose kernels overlap on
  *     the GPU (different streams, or graphs replayed concurrently) race.
+ *   - After wq_get_device_error has reported WQ_ERR_TIMEOUT on a device, the
+ *     next call there first clears the block's flags (cudaMemsetAsync on its
+ *     stream), since a timed-out call can leave one set.
  *   - A device with more SMs than the block has room for gets
  *     WQ_ERR_UNSUPPORTED, as does a workspace larger than the block.
  * Results are bit-identical to wq_matmul given a workspace. */

@@ -82,8 +82,19 @@ class Oracle:
         lib.oracle_half_round_up.restype = ctypes.c_uint16
         lib.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
         lib.oracle_bf16_to_double.restype = ctypes.c_double
+        lib.oracle_set_threads.argtypes = [ctypes.c_int]
+        lib.oracle_set_threads.restype = None
+        lib.oracle_max_threads.argtypes = []
+        lib.oracle_max_threads.restype = ctypes.c_int
         self.lib = lib
         self.path = path
+
+    def set_threads(self, n: int) -> None:
+        """Threads of the OpenMP loops (timing only; no effect on results)."""
+        self.lib.oracle_set_threads(int(n))
+
+    def max_threads(self) -> int:
+        return int(self.lib.oracle_max_threads())
 
     # -- quantize ----------------------------------------------------------
     def quantize(self, W_half_bits: np.ndarray, bits: int, group: int,

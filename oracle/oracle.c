@@ -40,6 +40,7 @@
  * Build: gcc -O2 -fopenmp -ffp-contract=off -fno-fast-math -shared -fPIC.
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <string.h>
 
@@ -419,3 +420,8 @@ void oracle_q4k_dequantize(const uint8_t *blocks, int64_t N, int64_t K, double *
 double oracle_half_to_double(uint16_t h) { return half_bits_to_double(h); }
 uint16_t oracle_half_round_up(double x) { return half_round_up_positive(x); }
 double oracle_bf16_to_double(uint16_t b) { return bf16_bits_to_double(b); }
+
+/* Thread count of the OpenMP loops above (timing the oracle at one thread
+ * and at all threads); not part of the arithmetic. */
+void oracle_set_threads(int n) { omp_set_num_threads(n > 0 ? n : 1); }
+int oracle_max_threads(void) { return omp_get_max_threads(); }

@@ -108,11 +108,22 @@ def _stream(device: torch.device):
 
 
 def _require_cuda(*tensors):
+    """Every tensor given is a contiguous CUDA tensor, all on one device; the
+    library runs on the current device, so calls are made with that device
+    current (``torch.cuda.device``)."""
+    device = None
     for t in tensors:
-        if t is not None and not t.is_cuda:
+        if t is None:
+            continue
+        if not t.is_cuda:
             raise ValueError("tensor must be on a CUDA device")
-        if t is not None and not t.is_contiguous():
+        if not t.is_contiguous():
             raise ValueError("tensor must be contiguous")
+        if device is None:
+            device = t.device
+        elif t.device != device:
+            raise ValueError(f"tensors on different devices: {device} and {t.device}")
+    return device
 
 
 def codes_bytes(N: int, K: int, bits: int) -> int:
@@ -160,9 +171,10 @@ def quantize(W: torch.Tensor, bits: int = 4, group: int = 128, symmetric: bool =
             scales=torch.empty((N, ne // N), dtype=torch.float16, device=dev),
             zeros=None if symmetric else torch.empty((N, ne // N), dtype=torch.float16, device=dev),
             N=N, K=K, bits=bits, group=group, symmetric=symmetric)
-    _require_cuda(out.codes, out.scales, out.zeros)
-    _check(lib.wq_quantize(_ptr(W), N, K, bits, group, int(symmetric), _ptr(out.codes),
-                           _ptr(out.scales), _ptr(out.zeros), _stream(W.device)), "wq_quantize")
+    dev = _require_cuda(W, out.codes, out.scales, out.zeros)
+    with torch.cuda.device(dev):
+        _check(lib.wq_quantize(_ptr(W), N, K, bits, group, int(symmetric), _ptr(out.codes),
+                               _ptr(out.scales), _ptr(out.zeros), _stream(dev)), "wq_quantize")
     return out
 
 
@@ -171,10 +183,11 @@ def dequantize(qw: QuantizedWeight, out: torch.Tensor | None = None) -> torch.Te
     _require_cuda(qw.codes, qw.scales, qw.zeros)
     if out is None:
         out = torch.empty((qw.N, qw.K), dtype=torch.bfloat16, device=qw.codes.device)
-    _require_cuda(out)
-    _check(lib.wq_dequantize(_ptr(qw.codes), _ptr(qw.scales), _ptr(qw.zeros), qw.N, qw.K,
-                             qw.bits, qw.group, int(qw.symmetric), _ptr(out),
-                             _stream(qw.codes.device)), "wq_dequantize")
+    dev = _require_cuda(qw.codes, qw.scales, qw.zeros, out)
+    with torch.cuda.device(dev):
+        _check(lib.wq_dequantize(_ptr(qw.codes), _ptr(qw.scales), _ptr(qw.zeros), qw.N, qw.K,
+                                 qw.bits, qw.group, int(qw.symmetric), _ptr(out),
+                                 _stream(dev)), "wq_dequantize")
     return out
 
 
@@ -215,15 +228,16 @@ def matmul(X: torch.Tensor, qw: QuantizedWeight, out_dtype: torch.dtype = torch.
     M = Xd.shape[0]
     Yd = out if (out is not None and out.is_cuda) else torch.empty(
         (M, qw.N), dtype=out_dtype, device=dev)
-    _require_cuda(Yd)
+    _require_cuda(Xd, qw.codes, qw.scales, qw.zeros, Yd)
     stream = torch.cuda.current_stream(dev).cuda_stream
     ws = workspace(dev, stream) if use_workspace else None
-    _check(lib.wq_matmul(_ptr(Xd), M, _ptr(qw.codes), _ptr(qw.scales), _ptr(qw.zeros), qw.N,
-                         qw.K, qw.bits, qw.group, int(qw.symmetric), _ptr(Yd),
-                         WQ_OUT_BF16 if Yd.dtype == torch.bfloat16 else WQ_OUT_F32,
-                         _ptr(ws), 0 if ws is None else ws.numel(),
-                         WQ_MATMUL_STATIC_WEIGHTS if static_weights else 0,
-                         ctypes.c_void_p(stream)), "wq_matmul")
+    with torch.cuda.device(dev):
+        _check(lib.wq_matmul(_ptr(Xd), M, _ptr(qw.codes), _ptr(qw.scales), _ptr(qw.zeros), qw.N,
+                             qw.K, qw.bits, qw.group, int(qw.symmetric), _ptr(Yd),
+                             WQ_OUT_BF16 if Yd.dtype == torch.bfloat16 else WQ_OUT_F32,
+                             _ptr(ws), 0 if ws is None else ws.numel(),
+                             WQ_MATMUL_STATIC_WEIGHTS if static_weights else 0,
+                             ctypes.c_void_p(stream)), "wq_matmul")
     if not host:
         return Yd
     if out is not None and not out.is_cuda:
@@ -248,8 +262,9 @@ def q4k_quantize(W: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tens
         raise WQError(1, "wq_q4k_quantize")
     if out is None:
         out = torch.empty((N, nb // N), dtype=torch.uint8, device=W.device)
-    _require_cuda(W, out)
-    _check(lib.wq_q4k_quantize(_ptr(W), N, K, _ptr(out), _stream(W.device)), "wq_q4k_quantize")
+    dev = _require_cuda(W, out)
+    with torch.cuda.device(dev):
+        _check(lib.wq_q4k_quantize(_ptr(W), N, K, _ptr(out), _stream(dev)), "wq_q4k_quantize")
     return out
 
 
@@ -264,10 +279,11 @@ def q4k_matmul(X: torch.Tensor, blocks: torch.Tensor, N: int, K: int,
         raise ValueError("out_dtype must be float32 or bfloat16")
     M = X.shape[0]
     Y = out if out is not None else torch.empty((M, N), dtype=out_dtype, device=X.device)
-    _require_cuda(X, blocks, Y)
-    _check(lib.wq_q4k_matmul(_ptr(X), M, _ptr(blocks), N, K, _ptr(Y),
-                             WQ_OUT_BF16 if Y.dtype == torch.bfloat16 else WQ_OUT_F32,
-                             _stream(X.device)), "wq_q4k_matmul")
+    dev = _require_cuda(X, blocks, Y)
+    with torch.cuda.device(dev):
+        _check(lib.wq_q4k_matmul(_ptr(X), M, _ptr(blocks), N, K, _ptr(Y),
+                                 WQ_OUT_BF16 if Y.dtype == torch.bfloat16 else WQ_OUT_F32,
+                                 _stream(dev)), "wq_q4k_matmul")
     return Y
 
 
@@ -281,16 +297,20 @@ def matmul_noalloc(X: torch.Tensor, qw: QuantizedWeight, out_dtype: torch.dtype 
     dev = qw.codes.device
     M = X.shape[0]
     Y = out if out is not None else torch.empty((M, qw.N), dtype=out_dtype, device=dev)
-    _require_cuda(Y)
-    _check(lib.wq_matmul_noalloc(_ptr(X), M, _ptr(qw.codes), _ptr(qw.scales), _ptr(qw.zeros),
-                                 qw.N, qw.K, qw.bits, qw.group, int(qw.symmetric), _ptr(Y),
-                                 WQ_OUT_BF16 if Y.dtype == torch.bfloat16 else WQ_OUT_F32,
-                                 WQ_MATMUL_STATIC_WEIGHTS if static_weights else 0,
-                                 _stream(dev)), "wq_matmul_noalloc")
+    _require_cuda(X, qw.codes, qw.scales, qw.zeros, Y)
+    # the library's scratch block is looked up on the current device
+    with torch.cuda.device(dev):
+        _check(lib.wq_matmul_noalloc(_ptr(X), M, _ptr(qw.codes), _ptr(qw.scales),
+                                     _ptr(qw.zeros), qw.N, qw.K, qw.bits, qw.group,
+                                     int(qw.symmetric), _ptr(Y),
+                                     WQ_OUT_BF16 if Y.dtype == torch.bfloat16 else WQ_OUT_F32,
+                                     WQ_MATMUL_STATIC_WEIGHTS if static_weights else 0,
+                                     _stream(dev)), "wq_matmul_noalloc")
     return Y
 
 
 def get_device_error(device: torch.device | None = None) -> int:
     """``wq_get_device_error``: read and clear the device status word."""
     device = device or torch.device("cuda", torch.cuda.current_device())
-    return lib.wq_get_device_error(_stream(device))
+    with torch.cuda.device(device):
+        return lib.wq_get_device_error(_stream(device))

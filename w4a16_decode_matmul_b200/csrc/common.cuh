@@ -13,7 +13,8 @@ namespace wq {
 
 // Device status word: 0 = fine; otherwise a wq_status code recorded by a
 // kernel (first writer wins).  Read and cleared by wq_get_device_error().
-__device__ unsigned int g_status;
+// Defined once, in wq.cu (the library is linked as relocatable device code).
+extern __device__ unsigned int g_status;
 
 // A wait gives up after this many nanoseconds of wall time (globaltimer).
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s

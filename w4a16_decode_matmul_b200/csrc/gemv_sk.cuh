@@ -93,6 +93,13 @@ struct Params {
   uint32_t stage_bytes;     // codes, scale blocks, zero blocks
   uint32_t off_ring, off_x, off_sx, off_red;
   uint32_t x_stride;        // bytes per staged activation row
+  // Test hooks of the timeout path (set only through an internal export):
+  // the CTA that does not publish its split-tile flag (-1: none), and the
+  // limit of the wait for published flags, in nanoseconds.  That wait comes
+  // after every copy and product of the waiting CTA has completed, so giving
+  // up there leaves nothing in flight.
+  int test_skip_publish;
+  unsigned long long flag_wait_ns;
 };
 
 struct Stage {
@@ -151,6 +158,21 @@ __host__ __device__ __forceinline__ void for_each_stage(int c, const Params& p, 
     while (!wk.done()) {
       const Stage st = wk.next(p.nk);
       fn(st, st.s1 == p.nk || wk.done());
+    }
+  }
+}
+
+// Wait until *flag == 1; false (and the status word set to WQ_ERR_TIMEOUT)
+// after limit_ns of wall time.
+__device__ __forceinline__ bool wait_flag_for(const unsigned int* flag,
+                                              unsigned long long limit_ns) {
+  if (ld_acquire_gpu(flag) == 1u) return true;
+  const unsigned long long start = global_timer_ns();
+  while (true) {
+    if (ld_acquire_gpu(flag) == 1u) return true;
+    if (global_timer_ns() - start > limit_ns) {
+      record_status(kStatusTimeout);
+      return false;
     }
   }
 }
@@ -477,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int o = lane; o < per_tile; o += 32)
         __stcg(p.ws_part + size_t(cta) * kWsRowsMax + o, warp_sum(li, o));
       __syncwarp();
-      if (lane == 0) st_release_gpu(p.ws_flag + cta, 1u);
+      if (lane == 0 && cta != p.test_skip_publish) st_release_gpu(p.ws_flag + cta, 1u);
       return;
     }
     // finish: own partial plus those of the CTAs whose (non-empty) tail
@@ -498,7 +520,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool pub = in && tail_begin(c2 + 1, p) > b2;
       const unsigned int in_mask = __ballot_sync(0xffffffffu, in);
       if (in_mask == 0u) break;
-      const bool ok = !pub || (*abort_flag == 0 && wait_flag(p.ws_flag + c2));
+      const bool ok = !pub || (*abort_flag == 0 && wait_flag_for(p.ws_flag + c2, p.flag_wait_ns));
       if (__ballot_sync(0xffffffffu, !ok) != 0u) {
         *abort_flag = 1;
         break;
