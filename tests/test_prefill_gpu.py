@@ -4,7 +4,13 @@ binary64 product of X and the oracle-dequantized weights:
 ulp for bfloat16 out.  Full outputs at reduced sizes that span several
 tiles and ragged M/N tails; sampled outputs (computed one by one by the
 oracle) at the full prefill sizes M in {512, 2048, 8192}, K=4096, N=14336;
-one-hot activations bit-exact (each output is one exact product s (q - z))."""
+one-hot activations bit-exact (each output is one exact product s (q - z)).
+Every test runs on both prefill kernels: the one with both operands in
+shared memory ("shared", groups of 64 or 128 with a multiple of 8 groups per
+row) and the one with the dequantized weights in tensor memory ("tmem",
+every group size, K a multiple of 64)."""
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -14,6 +20,23 @@ import synth
 from tests.gpu_util import check_tolerance, host_bits, oracle_quantize, weight, wq
 
 pytestmark = pytest.mark.gpu
+
+KERNELS = {"shared": 1, "tmem": 2}
+
+
+@pytest.fixture(params=sorted(KERNELS), autouse=True)
+def kernel(request):
+    lib = wq().lib
+    lib.wq_internal_set_prefill.argtypes = [ctypes.c_int]
+    lib.wq_internal_set_prefill(KERNELS[request.param])
+    yield request.param
+    lib.wq_internal_set_prefill(0)
+
+
+def in_scope(kernel, K, group):
+    if kernel == "shared":
+        return group in (64, 128) and (K // group) % 8 == 0 and K // group <= 256
+    return K % 64 == 0
 
 
 def quantize_both(W, bits, group, sym, key=None):
@@ -27,12 +50,15 @@ def quantize_both(W, bits, group, sym, key=None):
 
 
 @pytest.mark.parametrize("bits,group,sym", [(4, 128, False), (4, 64, True), (8, 128, False),
-                                            (8, 64, True), (4, 64, False), (8, 128, True)])
+                                            (8, 64, True), (4, 64, False), (8, 128, True),
+                                            (4, 32, False), (8, 32, True), (4, 32, True)])
 @pytest.mark.parametrize("M,N,K", [(33, 130, 1024), (128, 256, 1024), (200, 300, 2048),
-                                   (300, 1000, 512), (256, 128, 4096)])
-def test_reduced_sizes_full_outputs(M, N, K, bits, group, sym):
-    if (K // group) % 8:
-        pytest.skip("the prefill kernel takes a multiple of 8 groups per row")
+                                   (300, 1000, 512), (256, 128, 4096), (129, 257, 384)])
+def test_reduced_sizes_full_outputs(kernel, M, N, K, bits, group, sym):
+    if K % group:
+        pytest.skip("K is not a multiple of the group")
+    if not in_scope(kernel, K, group):
+        pytest.skip(f"outside the {kernel} prefill kernel's scope")
     W = synth.weight(N, K, seed=N + K + 1)
     X = synth.activation(M, K, seed=M + 7)
     qw, codes, scales, zeros = quantize_both(W, bits, group, sym)
@@ -67,8 +93,10 @@ def test_prefill_sizes_sampled(M):
     check_tolerance(Y.cpu().numpy()[ms, ns], y_ref, y_abs, False)
 
 
-@pytest.mark.parametrize("bits,group,sym", [(4, 128, False), (8, 64, True)])
-def test_one_hot_and_zero_activations_exact(bits, group, sym):
+@pytest.mark.parametrize("bits,group,sym", [(4, 128, False), (8, 64, True), (4, 32, False)])
+def test_one_hot_and_zero_activations_exact(kernel, bits, group, sym):
+    if not in_scope(kernel, 2048, group):
+        pytest.skip(f"outside the {kernel} prefill kernel's scope")
     N, K = 384, 2048
     W = synth.weight(N, K, seed=5)
     qw, codes, scales, zeros = quantize_both(W, bits, group, sym)
@@ -82,12 +110,13 @@ def test_one_hot_and_zero_activations_exact(bits, group, sym):
     assert np.all(Z == 0)
 
 
-def test_deterministic_and_out_of_scope():
+def test_deterministic_and_out_of_scope(kernel):
     N, K = 512, 4096
     qw = wq().quantize(synth.weight(N, K, seed=9).cuda())
     X = synth.activation(300, K, seed=10).cuda()
     assert torch.equal(wq().matmul(X, qw), wq().matmul(X, qw))
-    q32 = wq().quantize(synth.weight(N, K, seed=9).cuda(), group=32)
-    with pytest.raises(wq().WQError) as e:
-        wq().matmul(X, q32)
-    assert e.value.status == 2     # group 32 is outside the prefill kernel's scope
+    if kernel == "shared":
+        q32 = wq().quantize(synth.weight(N, K, seed=9).cuda(), group=32)
+        with pytest.raises(wq().WQError) as e:
+            wq().matmul(X, q32)
+        assert e.value.status == 2     # group 32 is outside this kernel's scope

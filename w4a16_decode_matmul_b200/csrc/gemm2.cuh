@@ -1,0 +1,482 @@
+// gemm2.cuh -- prefill-sized matmul Y = X * What^T (M > 32) on the fifth
+// generation tensor cores, weights as the tensor-memory operand: "vLLM 量化与
+// 推测解码" section 2 (W4A16: packed weights and group scales dequantized on
+// chip, multiplied with 16-bit activations, accumulated in higher precision)
+// and "量化" (llminference s08) section 实现 (large batches are bound by the
+// multiply: the weights are dequantized in on-chip tiles that feed the
+// tensor cores).
+//
+// Exactness: the tensor cores multiply the exact integers (q - z) (bfloat16
+// holds them) by the activations, one group at a time, into a binary32
+// accumulator D_g; y = sum_g s_g D_g is formed in binary32.  Products are
+// exact; only the binary32 sums round.
+//
+// Orientation (the transpose of Y is computed): the MMA's M dimension is 128
+// rows of W, its N dimension 128 tokens (rows of X), K runs along the
+// reduction.  A -- the dequantized weights -- lives in tensor memory,
+// written there by the dequantize warps with tcgen05.st, so the weight tile
+// never passes through shared memory; only the activation tile (B, from
+// shared memory, loaded by TMA) and the packed codes do.  Per 16 k step the
+// shared-memory traffic is the activation tile read by the MMA and written by
+// TMA plus the codes, about half that of a kernel with both operands in
+// shared memory.
+//
+// Persistent CTAs walk 128 x 128 tiles (token tile major, so that the CTAs of
+// a wave share one activation tile and the whole weight matrix stays in L2).
+// A load stage is 64 k: the activation box (128 tokens x 64 k, 128-byte
+// swizzle, K-major) and the codes box (128 rows x 64 k of codes, swizzled).
+// Warp roles:
+//   warp 0      TMA producer (one thread);
+//   warp 1      tensor-memory allocation; one thread issues tcgen05.mma
+//               (M=128, N=128, K=16) per 16 k from A in tensor memory and B
+//               in shared memory, into one of two 128-column group
+//               accumulators, and commits it to the epilogue after a group;
+//   warps 2-5   dequantize: one row of W per thread; a stage's codes ->
+//               32 columns of bfloat16 pairs (q - z) -> tensor memory
+//               (one of eight 32-column A stages);
+//   warps 6-13  epilogue: one row of W and 64 tokens per thread; per group
+//               S += s_g D_g in registers; S is written to Y at the end of
+//               the tile.
+// Every wait is bounded in time; a timeout records WQ_ERR_TIMEOUT, sets the
+// CTA's abort flag, the roles stop, issued copies and MMAs are drained and
+// tensor memory is freed.
+#pragma once
+
+#include "common.cuh"
+#include "gemm.cuh"
+
+namespace wq {
+namespace gemm2 {
+
+using gemm::fence_async_shared;
+using gemm::tc_commit;
+using gemm::tc_fence_after;
+using gemm::tc_fence_before;
+using gemm::tmem_ld32;
+using gemm::tmem_wait_ld;
+using gemm::umma_desc_sw128;
+
+constexpr int kBW = 128;     // rows of W per tile (MMA M)
+constexpr int kBT = 128;     // tokens per tile (MMA N)
+constexpr int kBK = 64;      // k per load stage
+constexpr int kMaxLoadStages = 8;
+constexpr int kAStages = 8;  // 32-column A stages in tensor memory
+constexpr int kDequantWarp0 = 2;
+constexpr int kNumEpilogueWarps = 8;
+// threads of a CTA with DW dequantize warps: producer, MMA, dequantize, epilogue
+constexpr int threads_for(int dw) { return (2 + dw + kNumEpilogueWarps) * 32; }
+constexpr int kXStageBytes = kBT * kBK * 2;                          // 16 KB
+constexpr int kTmemCols = 512;
+constexpr int kDCols = kBT;                       // one group accumulator
+constexpr int kACol0 = 2 * kDCols;                // A stages after the two accumulators
+constexpr int kAStageCols = kBK / 2;              // 64 k of bfloat16 pairs
+constexpr int kEpiCols = kBT / 2;                 // tokens per epilogue thread
+
+// mbarrier slots (8 bytes each) in the first KB of shared memory
+constexpr int kBarFull = 0;                    // [kMaxLoadStages] X + codes landed (tx)
+constexpr int kBarEmpty = 8;                   // [kMaxLoadStages] MMAs + dequantize done
+constexpr int kBarAFull = 16;                  // [kAStages] A stage written
+constexpr int kBarAEmpty = 24;                 // [kAStages] A stage read by the MMAs
+constexpr int kBarDFull = 32;                  // [2] group accumulator ready
+constexpr int kBarDEmpty = 34;                 // [2] group accumulator read
+constexpr int kBarMmaDone = 36;                // every MMA of the CTA finished
+constexpr int kTmemSlot = 512;                 // byte offset of the TMEM base address
+constexpr int kAbortSlot = 516;                // byte offset of the abort flag
+constexpr int kSmemHead = 1024;
+
+struct Params {
+  __nv_bfloat16* Y_bf16;   // one of Y_bf16 / Y_f32 is set
+  float* Y_f32;
+  const __half* scales;    // [N][ngroups]
+  const __half* zeros;     // [N][ngroups] (asymmetric)
+  int M, N, K, ngroups;
+  int tiles_t, tiles_w, num_tiles;
+  uint32_t codes_stage_bytes;  // kBW * kBK * bits / 8
+  uint32_t off_x, off_codes;   // rings (1024-byte aligned)
+};
+
+// A in tensor memory (M = 128 lanes, K = 16 as eight 32-bit columns of
+// bfloat16 pairs), B from a shared-memory descriptor.
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+      :
+      : "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(gemm::kInstrDesc), "r"(accumulate)
+      : "memory");
+}
+
+// 32 consecutive 32-bit columns of this warp's 32 lanes from registers.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31, %32};"
+      ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+      "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]),
+      "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]),
+      "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+      "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+
+// 16 consecutive 32-bit columns of this warp's 32 lanes from registers.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};"
+      ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+      "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]),
+      "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
+// 16 consecutive binary32 columns of this warp's 32 TMEM lanes.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// Eight 4-bit codes of a word (k = 0..7) -> four bfloat16 pairs in k order,
+// (u0-z, u1-z), (u2-z, u3-z), (u4-z, u5-z), (u6-z, u7-z); zb2 holds 128 + z
+// in both halves (the codes enter as the exact bfloat16 128 + u).
+__device__ __forceinline__ void dq4(uint32_t w, uint32_t zb2, uint32_t* o) {
+  constexpr uint32_t kMask = 0x000F000Fu, kMagic = 0x43004300u;
+  uint32_t t[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t r;
+    asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(r) : "r"(w >> (4 * i)), "r"(kMask), "r"(kMagic));
+    t[i] = r;  // (128 + u_i, 128 + u_{i+4})
+  }
+  o[0] = bf16x2_sub(__byte_perm(t[0], t[1], 0x5410), zb2);
+  o[1] = bf16x2_sub(__byte_perm(t[2], t[3], 0x5410), zb2);
+  o[2] = bf16x2_sub(__byte_perm(t[0], t[1], 0x7632), zb2);
+  o[3] = bf16x2_sub(__byte_perm(t[2], t[3], 0x7632), zb2);
+}
+
+// Four 8-bit codes -> two bfloat16 pairs (u0 - z, u1 - z), (u2 - z, u3 - z):
+// 2^23 + u in binary32 minus 2^23 + z is exact, and so is the conversion of
+// the integer (|u - z| < 256) to bfloat16.
+__device__ __forceinline__ void dq8(uint32_t w, float z, uint32_t* o) {
+  float f[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    f[i] = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7650 | i)) - (8388608.0f + z);
+  const __nv_bfloat162 p0 = __floats2bfloat162_rn(f[0], f[1]);
+  const __nv_bfloat162 p1 = __floats2bfloat162_rn(f[2], f[3]);
+  o[0] = *reinterpret_cast<const uint32_t*>(&p0);
+  o[1] = *reinterpret_cast<const uint32_t*>(&p1);
+}
+
+// LS: load stages in the shared-memory ring; DW: dequantize warps (4: one
+// per tensor-memory lane quarter, a whole stage each; 8: two per quarter,
+// half of a stage's k each).
+template <int BITS, bool SYM, int G, int LS, int DW>
+__global__ void __launch_bounds__(threads_for(DW), 1)
+    gemm2_kernel(const __grid_constant__ CUtensorMap tm_x,
+                 const __grid_constant__ CUtensorMap tm_codes, const Params p) {
+  static_assert(G == 32 || G == 64 || G == 128, "group");
+  static_assert(LS >= 2 && LS <= kMaxLoadStages && (DW == 4 || DW == 8), "roles");
+  constexpr int kLoadStages = LS;
+  constexpr int kNumDequantWarps = DW;
+  constexpr int kEpilogueWarp0 = kDequantWarp0 + DW;
+  constexpr int kStepsPerGroup = G / 16;        // 16-k MMA steps per group
+  constexpr int kCodesRowBytes = kBK * BITS / 8;  // 32 | 64 bytes of a row per stage
+  constexpr int kChunks = kCodesRowBytes / 16;     // 2 | 4 chunks of 16 bytes
+  constexpr int kMyChunks = kChunks * 4 / DW;      // chunks of a row per dequantize thread
+  constexpr int kMyCols = kAStageCols * 4 / DW;    // A columns per dequantize thread
+
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + kTmemSlot);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kAbortSlot);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int nkb = p.K / kBK;  // load stages per tile
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kLoadStages; ++s) {
+      mbar_init(&bars[kBarFull + s], 1);
+      mbar_init(&bars[kBarEmpty + s], 1 + kNumDequantWarps);
+    }
+    for (int s = 0; s < kAStages; ++s) {
+      mbar_init(&bars[kBarAFull + s], kNumDequantWarps);
+      mbar_init(&bars[kBarAEmpty + s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars[kBarDFull + b], 1);
+      mbar_init(&bars[kBarDEmpty + b], kNumEpilogueWarps);
+    }
+    mbar_init(&bars[kBarMmaDone], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(smem + kTmemSlot)),
+                 "r"(uint32_t(kTmemCols))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  auto wait = [&](int bar, uint32_t parity) {
+    if (*abort_flag) return false;
+    if (!mbar_wait(&bars[bar], parity)) {
+      *abort_flag = 1;
+      return false;
+    }
+    return true;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&tm_x);
+      prefetch_tensormap(&tm_codes);
+      const uint64_t keep = l2_policy_evict_last();  // both operands are reread by other CTAs
+      int issued = 0;
+      bool stop = false;
+      for (int tile = blockIdx.x; tile < p.num_tiles && !stop; tile += gridDim.x) {
+        const int t0 = (tile / p.tiles_w) * kBT, w0 = (tile % p.tiles_w) * kBW;
+        for (int kb = 0; kb < nkb; ++kb, ++issued) {
+          const int s = issued % kLoadStages;
+          const uint32_t ph = uint32_t(issued / kLoadStages) & 1u;
+          if (!wait(kBarEmpty + s, ph ^ 1u)) {
+            stop = true;
+            break;
+          }
+          mbar_arrive_expect_tx(&bars[kBarFull + s], uint32_t(kXStageBytes) + p.codes_stage_bytes);
+          tma_load_2d(smem + p.off_x + s * kXStageBytes, &tm_x, &bars[kBarFull + s], kb * kBK,
+                      t0, keep);
+          tma_load_2d(smem + p.off_codes + s * p.codes_stage_bytes, &tm_codes,
+                      &bars[kBarFull + s], kb * kCodesRowBytes, w0, keep);
+        }
+      }
+      // every issued copy lands before the CTA can finish
+      for (int j = max(0, issued - kLoadStages); j < issued; ++j)
+        mbar_wait(&bars[kBarFull + j % kLoadStages], uint32_t(j / kLoadStages) & 1u);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t xs0 = smem_addr(smem + p.off_x);
+      int ld = 0;       // load stages consumed
+      int gcount = 0;   // groups accumulated (selects the D buffer)
+      bool stop = false;
+      for (int tile = blockIdx.x; tile < p.num_tiles && !stop; tile += gridDim.x) {
+        int step_in_group = 0;
+        uint32_t d = 0;
+        for (int kb = 0; kb < nkb && !stop; ++kb, ++ld) {
+          const int s = ld % kLoadStages;
+          const int as = ld % kAStages;
+          if (!wait(kBarFull + s, uint32_t(ld / kLoadStages) & 1u) ||
+              !wait(kBarAFull + as, uint32_t(ld / kAStages) & 1u)) {
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t xdesc = umma_desc_sw128(xs0 + uint32_t(s) * kXStageBytes);
+          const uint32_t a_addr = tmem_base + uint32_t(kACol0 + as * kAStageCols);
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            if (step_in_group == 0) {
+              const int db = gcount & 1;
+              if (!wait(kBarDEmpty + db, (uint32_t(gcount >> 1) & 1u) ^ 1u)) {
+                stop = true;
+                break;
+              }
+              tc_fence_after();
+              d = tmem_base + uint32_t(db * kDCols);
+            }
+            tc_mma_ts(d, a_addr + uint32_t(8 * k), xdesc + uint64_t(2 * k),
+                      step_in_group > 0 ? 1u : 0u);
+            if (++step_in_group == kStepsPerGroup) {
+              tc_commit(&bars[kBarDFull + (gcount & 1)]);
+              step_in_group = 0;
+              ++gcount;
+            }
+          }
+          if (stop) break;
+          // the stage's activations and A columns are free once these MMAs finish
+          tc_commit(&bars[kBarEmpty + s]);
+          tc_commit(&bars[kBarAEmpty + as]);
+        }
+      }
+      // all MMAs of this CTA complete before tensor memory is freed
+      tc_commit(&bars[kBarMmaDone]);
+      mbar_wait(&bars[kBarMmaDone], 0);
+    }
+  } else if (warp < kEpilogueWarp0) {
+    // ------------------------------------------------------------ dequantize
+    // one row of the weight tile per thread; the warp's lanes are its 32
+    // rows of tensor memory
+    const int quarter = warp & 3;
+    const int r = 32 * quarter + lane;  // row of the W tile = TMEM lane
+    const uint32_t lanes = uint32_t(32 * quarter) << 16;
+    const int part = (warp - kDequantWarp0) >> 2;  // which share of the stage's k (DW = 8)
+    int ld = 0;
+    bool stop = false;
+    for (int tile = blockIdx.x; tile < p.num_tiles && !stop; tile += gridDim.x) {
+      const int w0 = (tile % p.tiles_w) * kBW;
+      const int row = w0 + r;
+      const bool row_ok = row < p.N;
+      const __half* zrow = p.zeros + size_t(row_ok ? row : 0) * p.ngroups;
+      for (int kb = 0; kb < nkb; ++kb, ++ld) {
+        const int s = ld % kLoadStages;
+        const int as = ld % kAStages;
+        if (!wait(kBarFull + s, uint32_t(ld / kLoadStages) & 1u) ||
+            !wait(kBarAEmpty + as, (uint32_t(ld / kAStages) & 1u) ^ 1u)) {
+          stop = true;
+          break;
+        }
+        tc_fence_after();
+        // the stage's codes of row r, unswizzled: chunk c sits at chunk
+        // c ^ key (32-byte swizzle: bit 4 of the address XOR bit 7; 64-byte
+        // swizzle: bits 4-5 XOR bits 7-8)
+        const uint8_t* crow = smem + p.off_codes + s * p.codes_stage_bytes + r * kCodesRowBytes;
+        const int key = kChunks == 2 ? ((r >> 2) & 1) : ((r >> 1) & 3);
+        uint32_t o[kMyCols];
+        if constexpr (BITS == 4) {
+#pragma unroll
+          for (int cc = 0; cc < kMyChunks; ++cc) {  // 16 bytes = 32 k
+            const int c = part * kMyChunks + cc;
+            const uint4 v = *reinterpret_cast<const uint4*>(crow + ((c ^ key) << 4));
+            const int k0 = kb * kBK + 32 * c;
+            float zf = SYM ? 8.f : 0.f;
+            if (!SYM) zf = row_ok ? __half2float(zrow[k0 / G]) : 0.f;
+            const __nv_bfloat162 zz = __floats2bfloat162_rn(128.f + zf, 128.f + zf);
+            const uint32_t zb2 = *reinterpret_cast<const uint32_t*>(&zz);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) dq4(w[j], zb2, o + 16 * cc + 4 * j);
+          }
+        } else {
+#pragma unroll
+          for (int cc = 0; cc < kMyChunks; ++cc) {  // 16 bytes = 16 k
+            const int c = part * kMyChunks + cc;
+            const uint4 v = *reinterpret_cast<const uint4*>(crow + ((c ^ key) << 4));
+            const int k0 = kb * kBK + 16 * c;
+            float zf = SYM ? 128.f : 0.f;
+            if (!SYM) zf = row_ok ? __half2float(zrow[k0 / G]) : 0.f;
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) dq8(w[j], zf, o + 8 * cc + 2 * j);
+          }
+        }
+        if (!row_ok) {
+#pragma unroll
+          for (int i = 0; i < kMyCols; ++i) o[i] = 0u;
+        }
+        // the codes of this stage are consumed
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[kBarEmpty + s]);
+        const uint32_t col = uint32_t(kACol0 + as * kAStageCols + part * kMyCols);
+        if constexpr (kMyCols == 32) {
+          tmem_st32(tmem_base + lanes + col, o);
+        } else {
+          tmem_st16(tmem_base + lanes + col, o);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[kBarAFull + as]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int e = warp - kEpilogueWarp0;  // 0..7
+    const int quarter = warp & 3;         // TMEM lanes 32 * quarter ..
+    const int half = e >> 2;              // tokens 64 * half .. of the tile
+    const int r = 32 * quarter + lane;    // row of the W tile
+    const uint32_t lanes = uint32_t(32 * quarter) << 16;
+    int gcount = 0;
+    bool stop = false;
+    for (int tile = blockIdx.x; tile < p.num_tiles && !stop; tile += gridDim.x) {
+      const int t0 = (tile / p.tiles_w) * kBT, w0 = (tile % p.tiles_w) * kBW;
+      const int row = w0 + r;
+      const bool row_ok = row < p.N;
+      const __half* srow = p.scales + size_t(row_ok ? row : 0) * p.ngroups;
+      float S[kEpiCols];
+#pragma unroll
+      for (int j = 0; j < kEpiCols; ++j) S[j] = 0.f;
+      int done = 0;
+      for (int gi = 0; gi < p.ngroups; ++gi, ++gcount) {
+        const float sg = row_ok ? __half2float(srow[gi]) : 0.f;
+        const int db = gcount & 1;
+        if (!wait(kBarDFull + db, uint32_t(gcount >> 1) & 1u)) {
+          stop = true;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + lanes + uint32_t(db * kDCols + half * kEpiCols);
+        float dv[16];
+#pragma unroll
+        for (int h = 0; h < kEpiCols / 16; ++h) {
+          tmem_ld16(taddr + 16 * h, dv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) S[16 * h + j] = fmaf(sg, dv[j], S[16 * h + j]);
+        }
+        // D_g is read: the MMA warp may overwrite this buffer
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[kBarDEmpty + db]);
+        done = gi + 1;
+      }
+      if (stop || done != p.ngroups || *abort_flag) break;
+      if (row_ok) {
+        const int tb = t0 + half * kEpiCols;
+#pragma unroll
+        for (int j = 0; j < kEpiCols; ++j) {
+          const int m = tb + j;
+          if (m < p.M) {
+            if (p.Y_f32 != nullptr)
+              p.Y_f32[size_t(m) * p.N + row] = S[j];
+            else
+              p.Y_bf16[size_t(m) * p.N + row] = __float2bfloat16_rn(S[j]);
+          }
+        }
+      }
+    }
+  }
+
+  // tensor memory is freed by the warp that allocated it, after every reader
+  // and every MMA is done
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(uint32_t(kTmemCols))
+                 : "memory");
+  }
+}
+
+}  // namespace gemm2
+}  // namespace wq

@@ -19,11 +19,12 @@
 //     unit's row r (one instruction: rows 0-3, whole lines) and of row r + 4
 //     (a second one) into its own 32 bytes of a per-warp ring of DEPTH units
 //     in shared memory (cp.async: no registers held while in flight), and
-//     reads them back itself when the unit is computed.  The
-//     first DEPTH units are requested before the wait on the previous grid
-//     when the caller promises the weights are static.  The CTA's scales and
-//     zeros (a contiguous block of each tensor) are read once, coalesced,
-//     into a shared-memory table of binary32 pairs {s, 128 + z}.
+//     reads them back itself when the unit is computed.  The CTA's scales
+//     and zeros (a contiguous block of each tensor) are read once, coalesced,
+//     into a shared-memory table of binary32 pairs {s, 128 + z}.  When the
+//     caller promises the weights are static, the first DEPTH units, the
+//     table and the clearing of the partial sums all happen before the wait
+//     on the previous grid; only the activations are read after it.
 //   * Seen as mma.sync m16n8k16 fragments (lane = 4 g + t), lane L holds row
 //     g of the A operand with g = 2 r + (c / 4), i.e. A row g is (tile row
 //     g / 2, group g % 2 of the pair) and rows g + 8 are tile rows 4 + g / 2.
@@ -52,12 +53,12 @@ namespace ld {
 
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
-constexpr int kDepth = 3;        // units in flight per warp (shared-memory ring)
+constexpr int kDepth = 3;        // default units in flight per warp (shared-memory ring)
+constexpr int kMaxDepth = 8;
 constexpr int kMaxM = 4;
 constexpr int kGroup = 128;      // codes per group (4-bit: 64 bytes of a row)
 constexpr int kTileRows = 8;
 constexpr int kUnitBytes = 128;  // bytes of one tile row in a unit (a pair of groups)
-constexpr int kMetaRegs = 2;     // blocks of 4 scales (and zeros) per thread read early
 
 struct Params {
   const __nv_bfloat16* X;  // [M][K]
@@ -69,11 +70,15 @@ struct Params {
   int tiles;               // ceil(N / 8)
   int y_bf16;
   int pdl;                 // weights may be read before the previous grid completes
+  // 2^28, 2^24, 2^20: the high word of w times these is w >> 4, 8, 12.  Given
+  // as parameters (values the compiler cannot see), the right shifts of the
+  // unpack run as integer multiplies on the FMA pipe instead of the ALU pipe.
+  uint32_t mul_shr4, mul_shr8, mul_shr12;
   uint32_t xs_row_bytes;   // K * 2 + 64: shared-memory bytes per activation row
   uint32_t off_sx;         // [M][ngroups] binary32 group sums
   uint32_t off_sz;         // [rows of the CTA][ngroups + 1] {scale, 128 + zero} binary32
   uint32_t off_part;       // [tiles per CTA][kWarps][8][M] binary32 partials
-  uint32_t off_ring;       // [kWarps][kDepth][2][32 lanes][16 bytes] codes ring
+  uint32_t off_ring;       // [kWarps][DEPTH][2][32 lanes][16 bytes] codes ring
 };
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
@@ -96,6 +101,30 @@ __device__ __forceinline__ uint2 ldg_stream64(const void* p) {
                : "=r"(v.x), "=r"(v.y)
                : "l"(p));
   return v;
+}
+
+__device__ __forceinline__ uint32_t mul_hi(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.hi.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// Eight 4-bit codes of one word -> four bfloat16 pairs (128 + u), as
+// unpack_u4, with the three right shifts either on the ALU pipe (SHF) or as
+// multiplies by 2^(32-s) keeping the high word (the FMA pipe).
+template <bool FMA_SHIFT>
+__device__ __forceinline__ void unpack_u4_pipe(uint32_t w, uint32_t (&r)[4], const Params& p) {
+  constexpr uint32_t kMask = 0x000F000Fu, kMagic = 0x43004300u;  // bf16 128.0 pair
+  r[0] = lop3_and_or(w, kMask, kMagic);
+  if constexpr (FMA_SHIFT) {
+    r[1] = lop3_and_or(mul_hi(w, p.mul_shr4), kMask, kMagic);
+    r[2] = lop3_and_or(mul_hi(w, p.mul_shr8), kMask, kMagic);
+    r[3] = lop3_and_or(mul_hi(w, p.mul_shr12), kMask, kMagic);
+  } else {
+    r[1] = lop3_and_or(w >> 4, kMask, kMagic);
+    r[2] = lop3_and_or(w >> 8, kMask, kMagic);
+    r[3] = lop3_and_or(w >> 12, kMask, kMagic);
+  }
 }
 
 // The fetch side of a warp's units: the byte offset of this lane's 16 bytes
@@ -142,9 +171,12 @@ struct UnitWalk {
 };
 
 // MT: a compile-time bound on M (1, 2 or 4), so that lanes whose token
-// columns cannot exist keep no accumulators.
-template <bool SYM, int MT>
-__global__ void __launch_bounds__(kThreads, 1) gemv_ld_kernel(const Params p) {
+// columns cannot exist keep no accumulators.  DEPTH: units in flight per
+// warp.  FMA_SHIFT: the unpack's right shifts as multiplies (FMA pipe).
+// MINB: CTAs per SM the register allocation must allow (2 lets the next
+// launch's CTA start streaming while this one finishes).
+template <bool SYM, int MT, int DEPTH, bool FMA_SHIFT, int MINB>
+__global__ void __launch_bounds__(kThreads, MINB) gemv_ld_kernel(const Params p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = lane >> 3, c = lane & 7;  // load view: tile row r (and r + 4), chunk c
@@ -166,7 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_ld_kernel(const Params p) {
               size_t(c) * 16;
   fetch.set_rows(p.N);
   // this lane's 16 bytes of slot 0 (row r); slot j at + 1024 j
-  const uint32_t ring = smem_addr(smem) + p.off_ring + uint32_t(warp * kDepth * 1024 + lane * 16);
+  const uint32_t ring = smem_addr(smem) + p.off_ring + uint32_t(warp * DEPTH * 1024 + lane * 16);
   // one commit group per unit (empty past the end) keeps the wait count fixed
   auto prefetch = [&](int slot) {
     if (fetch.left > 0) {
@@ -176,41 +208,49 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_ld_kernel(const Params p) {
     cp_async_commit();
   };
 
-  // the CTA's scales and zeros: rows [8 tb0, min(N, 8 tb1)) x ngroups, as
-  // contiguous blocks of 4 binary16 values (ngroups is even, rows start at a
-  // multiple of 8: every block is 8-byte aligned and inside one row)
-  const int row_lo = tb0 * kTileRows;
-  const int rows = min(p.N, tb1 * kTileRows) - row_lo;
-  const int meta4 = rows * ng / 4;
-  uint2 sv[kMetaRegs], zv[kMetaRegs];
-  auto load_meta = [&]() {
-#pragma unroll
-    for (int j = 0; j < kMetaRegs; ++j) {
-      const int i = int(threadIdx.x) + j * kThreads;
-      sv[j] = zv[j] = make_uint2(0, 0);
-      if (i < meta4) {
-        sv[j] = ldg_stream64(p.scales + size_t(row_lo) * ng + 4 * size_t(i));
-        if (!SYM) zv[j] = ldg_stream64(p.zeros + size_t(row_lo) * ng + 4 * size_t(i));
-      }
-    }
-  };
-  if (p.pdl) {
-#pragma unroll
-    for (int j = 0; j < kDepth; ++j) prefetch(j);
-    load_meta();
-  }
-  grid_dependents_launch();
-  grid_dependency_wait();
-  if (!p.pdl) {
-#pragma unroll
-    for (int j = 0; j < kDepth; ++j) prefetch(j);
-    load_meta();
-  }
-
   float* sx = reinterpret_cast<float*>(smem + p.off_sx);
   float2* sz = reinterpret_cast<float2*>(smem + p.off_sz);
   float* part = reinterpret_cast<float*>(smem + p.off_part);
   const int sz_stride = ng + 1;  // entries per row: rows land on different banks
+
+  // The weight-side set-up, which reads no input the previous kernel may
+  // write: the first DEPTH units of every warp are requested, the CTA's
+  // scales and zeros -- rows [8 tb0, min(N, 8 tb1)) x ngroups, contiguous
+  // blocks of 4 binary16 values (ngroups is even and rows start at a
+  // multiple of 8: every block is 8-byte aligned and inside one row) -- are
+  // turned into the {s, 128 + z} table (symmetric: 128 + 8), and the partial
+  // sums are cleared.  With static weights all of this happens before the
+  // wait on the previous grid.
+  const int row_lo = tb0 * kTileRows;
+  const int rows = min(p.N, tb1 * kTileRows) - row_lo;
+  const int meta4 = rows * ng / 4;
+  auto weight_setup = [&]() {
+#pragma unroll
+    for (int j = 0; j < DEPTH; ++j) prefetch(j);
+    for (int i = int(threadIdx.x); i < meta4; i += kThreads) {
+      const uint2 a = ldg_stream64(p.scales + size_t(row_lo) * ng + 4 * size_t(i));
+      const uint2 z = SYM ? make_uint2(0, 0)
+                          : ldg_stream64(p.zeros + size_t(row_lo) * ng + 4 * size_t(i));
+      const int e = 4 * i, row = e / ng, gi = e - row * ng;
+      float2* d = sz + row * sz_stride + gi;
+      const uint32_t sw[2] = {a.x, a.y}, zw[2] = {z.x, z.y};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t sk = (sw[k >> 1] >> (16 * (k & 1))) & 0xFFFFu;
+        const uint32_t zk = (zw[k >> 1] >> (16 * (k & 1))) & 0xFFFFu;
+        const float bias =
+            SYM ? 136.f : 128.f + __half2float(__ushort_as_half(static_cast<unsigned short>(zk)));
+        d[k] = make_float2(__half2float(__ushort_as_half(static_cast<unsigned short>(sk))), bias);
+      }
+    }
+    const int nparts = (tb1 - tb0) * kWarps * kTileRows * p.M;
+    for (int i = threadIdx.x; i < nparts; i += kThreads) part[i] = 0.f;
+  };
+  if (p.pdl) weight_setup();
+  grid_dependents_launch();
+  grid_dependency_wait();
+  if (!p.pdl) weight_setup();
+
   {
     // activations, permuted, and their group sums
     const int total8 = p.M * p.K / 8;  // a multiple of 16: groups of 128 never straddle
@@ -239,34 +279,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_ld_kernel(const Params p) {
       for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
       if (ok && (threadIdx.x & 15) == 0) sx[(8 * i) / kGroup] = sum;  // [n][gi] flattened
     }
-    // scales and zeros as {s, 128 + z} (symmetric: 128 + 8): the blocks held
-    // in registers, then any further blocks of a large CTA share
-    auto store_meta = [&](int i, uint2 a, uint2 z) {
-      const int e = 4 * i, row = e / ng, gi = e - row * ng;
-      float2* d = sz + row * sz_stride + gi;
-      const uint32_t sw[2] = {a.x, a.y}, zw[2] = {z.x, z.y};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint32_t sk = (sw[k >> 1] >> (16 * (k & 1))) & 0xFFFFu;
-        const uint32_t zk = (zw[k >> 1] >> (16 * (k & 1))) & 0xFFFFu;
-        const float bias =
-            SYM ? 136.f : 128.f + __half2float(__ushort_as_half(static_cast<unsigned short>(zk)));
-        d[k] = make_float2(__half2float(__ushort_as_half(static_cast<unsigned short>(sk))), bias);
-      }
-    };
-#pragma unroll
-    for (int j = 0; j < kMetaRegs; ++j) {
-      const int i = int(threadIdx.x) + j * kThreads;
-      if (i < meta4) store_meta(i, sv[j], zv[j]);
-    }
-    for (int i = int(threadIdx.x) + kMetaRegs * kThreads; i < meta4; i += kThreads) {
-      const uint2 a = ldg_stream64(p.scales + size_t(row_lo) * ng + 4 * size_t(i));
-      const uint2 z = SYM ? make_uint2(0, 0)
-                          : ldg_stream64(p.zeros + size_t(row_lo) * ng + 4 * size_t(i));
-      store_meta(i, a, z);
-    }
-    const int nparts = (tb1 - tb0) * kWarps * kTileRows * p.M;
-    for (int i = threadIdx.x; i < nparts; i += kThreads) part[i] = 0.f;
   }
   __syncthreads();
 
@@ -313,14 +325,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_ld_kernel(const Params p) {
 
   while (use.left > 0) {
 #pragma unroll
-    for (int j = 0; j < kDepth; ++j) {
+    for (int j = 0; j < DEPTH; ++j) {
       if (use.left > 0) {
         if (use.tile != cur_tile) {
           flush();
           cur_tile = use.tile;
           sz0 = sz + ((cur_tile - tb0) * kTileRows + rr0) * sz_stride;
         }
-        cp_async_wait<kDepth - 1>();  // this unit's copies (issued by this lane) landed
+        cp_async_wait<DEPTH - 1>();  // this unit's copies (issued by this lane) landed
         const uint4 c0 = lds128(ring + uint32_t(j) * 1024);
         const uint4 c1 = lds128(ring + uint32_t(j) * 1024 + 512);
         const int pair = use.pair;
@@ -330,8 +342,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_ld_kernel(const Params p) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           uint32_t pa[4], pb[4];
-          unpack_u4(w0[q], pa);
-          unpack_u4(w1[q], pb);
+          unpack_u4_pipe<FMA_SHIFT>(w0[q], pa, p);
+          unpack_u4_pipe<FMA_SHIFT>(w1[q], pb, p);
           uint4 xv = make_uint4(0, 0, 0, 0);
           if (has_x) xv = lds128(xs_lane + (uint32_t(pair * 4 + q) << 7));
           const uint32_t a_even[4] = {pa[0], pb[0], pa[1], pb[1]};

@@ -78,6 +78,7 @@ bool run_ld(const MatmulArgs& a, cudaError_t* err);
 bool run_sk(const MatmulArgs& a, bool split, cudaError_t* err);
 bool run_gemv(const MatmulArgs& a, cudaError_t* err);
 bool run_gemm(const MatmulArgs& a, cudaError_t* err);
+bool run_gemm2(const MatmulArgs& a, cudaError_t* err);
 
 cudaError_t run_quantize(int bits, bool sym, int group, const void* W, int64_t total,
                          void* codes, void* scales, void* zeros, cudaStream_t s, int sms);
@@ -97,6 +98,11 @@ int sk_workspace_ctas();
 // the cluster-split kernel, 2 the balanced kernel, 3 the balanced kernel
 // with row tiles split across CTAs, 4 the direct-load kernel.
 extern int g_kernel_choice;
+
+// Prefill kernel for wq_matmul at M > 32 (tuning and test hook): 0 chooses
+// (the weights-in-tensor-memory kernel wherever it applies), 1 forces the
+// kernel with both operands in shared memory, 2 forces the former.
+extern int g_prefill_choice;
 
 // Calls every format the library supports through F<BITS, SYM, G>::run.
 template <template <int, bool, int> class F, typename... Args>

@@ -1,0 +1,148 @@
+// k_gemm2.cu -- plan and launch of the prefill matmul with the weights as
+// the tensor-memory operand (gemm2.cuh).
+#include <algorithm>
+
+#include "host.h"
+#include "gemm2.cuh"
+
+namespace wqh {
+namespace {
+
+struct Gemm2Plan {
+  wq::gemm2::Params p;
+  int grid = 1;
+  size_t smem = 0;
+  int variant = 0;
+};
+
+// Build variants (load stages, dequantize warps), chosen through an internal
+// tuning hook.
+struct Gemm2Variant {
+  int load_stages, dequant_warps;
+};
+constexpr Gemm2Variant kGemm2Variants[] = {{4, 4}, {8, 4}, {8, 8}, {6, 8}};
+constexpr int kNumGemm2Variants = int(sizeof(kGemm2Variants) / sizeof(kGemm2Variants[0]));
+int g_gemm2_variant = 0;
+
+// Scope: groups of 32, 64 or 128, K a multiple of 64; any M and N.
+bool plan_gemm2(int M, int N, int K, int bits, int group, const DeviceInfo& dev,
+                Gemm2Plan* plan, int variant) {
+  using namespace wq::gemm2;
+  if (variant < 0 || variant >= kNumGemm2Variants) return false;
+  plan->variant = variant;
+  const int stages = kGemm2Variants[variant].load_stages;
+  if (group != 32 && group != 64 && group != 128) return false;
+  if (bits != 4 && bits != 8) return false;
+  if (K % kBK != 0 || K % group != 0 || M < 1 || N < 1) return false;
+  wq::gemm2::Params& p = plan->p;
+  p = wq::gemm2::Params{};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.ngroups = K / group;
+  p.tiles_t = (M + kBT - 1) / kBT;
+  p.tiles_w = (N + kBW - 1) / kBW;
+  const long long tiles = (long long)p.tiles_t * p.tiles_w;
+  if (tiles > 0x7fffffffLL) return false;
+  p.num_tiles = int(tiles);
+  p.codes_stage_bytes = uint32_t(kBW * kBK * bits / 8);
+  p.off_x = kSmemHead;
+  p.off_codes = p.off_x + uint32_t(stages * kXStageBytes);
+  plan->smem = p.off_codes + size_t(stages) * p.codes_stage_bytes;
+  if (plan->smem > size_t(dev.max_smem_optin)) return false;
+  plan->grid = std::min(p.num_tiles, dev.sms);
+  return true;
+}
+
+template <int BITS, bool SYM, int G, int LS, int DW>
+cudaError_t launch_gemm2(Gemm2Plan* plan, const DeviceInfo* dev, const void* X, const void* c,
+                         cudaStream_t s) {
+  using namespace wq::gemm2;
+  auto kernel = &gemm2_kernel<BITS, SYM, G, LS, DW>;
+  static int configured[kMaxDevices] = {};
+  {
+    const cudaError_t e = configure_smem(kernel, configured, size_t(dev->max_smem_optin));
+    if (e != cudaSuccess) return e;
+  }
+  const wq::gemm2::Params& p = plan->p;
+  CUtensorMap tx, tc;
+  // X [M][K] bfloat16, boxes of 64 k x 128 tokens, 128-byte swizzle (the
+  // K-major canonical layout of the MMA's B operand)
+  if (!encode_2d_ex(&tx, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, uint64_t(p.K), uint64_t(p.M),
+                    uint32_t(kBK), uint32_t(kBT), CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
+    return cudaErrorInvalidValue;
+  // codes [N][K*bits/8] bytes, boxes of 64 k x 128 rows, swizzled so that
+  // the dequantize threads (one row each) read without bank conflicts
+  const uint32_t row_box = uint32_t(kBK * BITS / 8);
+  if (!encode_2d_ex(&tc, c, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(p.K) * BITS / 8,
+                    uint64_t(p.N), row_box, uint32_t(kBW),
+                    BITS == 4 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
+    return cudaErrorInvalidValue;
+  kernel<<<plan->grid, threads_for(DW), plan->smem, s>>>(tx, tc, p);
+  return cudaGetLastError();
+}
+
+template <int BITS, bool SYM, int G>
+struct Gemm2Op {
+  static cudaError_t run(Gemm2Plan* plan, const DeviceInfo* dev, const void* X, const void* c,
+                         cudaStream_t s) {
+    switch (plan->variant) {
+      case 1: return launch_gemm2<BITS, SYM, G, 8, 4>(plan, dev, X, c, s);
+      case 2: return launch_gemm2<BITS, SYM, G, 8, 8>(plan, dev, X, c, s);
+      case 3: return launch_gemm2<BITS, SYM, G, 6, 8>(plan, dev, X, c, s);
+      default: return launch_gemm2<BITS, SYM, G, 4, 4>(plan, dev, X, c, s);
+    }
+  }
+};
+
+}  // namespace
+
+bool run_gemm2(const MatmulArgs& a, cudaError_t* err) {
+  Gemm2Plan gp;
+  if (!plan_gemm2(a.M, a.N, a.K, a.bits, a.group, a.dev, &gp, g_gemm2_variant) &&
+      (g_gemm2_variant == 0 || !plan_gemm2(a.M, a.N, a.K, a.bits, a.group, a.dev, &gp, 0)))
+    return false;
+  if (a.y_bf16)
+    gp.p.Y_bf16 = static_cast<__nv_bfloat16*>(a.Y);
+  else
+    gp.p.Y_f32 = static_cast<float*>(a.Y);
+  gp.p.scales = static_cast<const __half*>(a.scales);
+  gp.p.zeros = static_cast<const __half*>(a.zeros);
+  *err = dispatch_format<Gemm2Op>(a.bits, a.sym, a.group, &gp, &a.dev, a.X, a.codes, a.stream);
+  return true;
+}
+
+}  // namespace wqh
+
+extern "C" {
+
+// Test hook, not part of the public ABI: the prefill plan with the weights in
+// tensor memory, written to out[0..9] (M, N, K, ngroups, tiles_t, tiles_w,
+// num_tiles, codes_stage_bytes, smem, grid).  Returns 0 if the shape is
+// outside the kernel's scope.
+int wq_internal_plan_gemm2(int M, int N, int K, int bits, int group, int sms, int smem_optin,
+                           int64_t* out) {
+  wqh::DeviceInfo dev;
+  dev.sms = sms;
+  dev.max_smem_optin = smem_optin;
+  wqh::Gemm2Plan plan;
+  if (!wqh::plan_gemm2(M, N, K, bits, group, dev, &plan, 0)) return 0;
+  const wq::gemm2::Params& p = plan.p;
+  const int64_t v[] = {p.M,         p.N,         p.K,         p.ngroups,         p.tiles_t,
+                       p.tiles_w,   p.num_tiles, p.codes_stage_bytes, int64_t(plan.smem),
+                       plan.grid};
+  for (size_t i = 0; i < sizeof(v) / sizeof(v[0]); ++i) out[i] = v[i];
+  return 1;
+}
+
+// Tuning hook, not part of the public ABI: the build variant of the prefill
+// kernel with the weights in tensor memory (0 .. 3, see kGemm2Variants; one
+// that does not fit falls back to 0).  Returns the number of variants.
+int wq_internal_set_gemm2_variant(int variant) {
+  if (variant >= 0 && variant < wqh::kNumGemm2Variants) wqh::g_gemm2_variant = variant;
+  return wqh::kNumGemm2Variants;
+}
+
+}  // extern "C"

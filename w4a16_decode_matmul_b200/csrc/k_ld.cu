@@ -12,7 +12,21 @@ struct LdPlan {
   wq::ld::Params p;
   int grid = 1;
   size_t smem = 0;
+  int variant = 0;
 };
+
+// Build variants of the kernel (ring depth, pipe of the unpack shifts, CTAs
+// per SM the registers must allow), chosen through an internal tuning hook.
+struct LdVariant {
+  int depth;
+  bool fma_shift;
+  int min_blocks;
+};
+constexpr LdVariant kLdVariants[] = {
+    {3, false, 1}, {3, true, 1}, {4, true, 2}, {6, true, 1}, {4, false, 2}, {6, false, 1},
+};
+constexpr int kNumLdVariants = int(sizeof(kLdVariants) / sizeof(kLdVariants[0]));
+int g_ld_variant = 0;
 
 // Plan the direct-load kernel: 4-bit codes in groups of 128 with K a
 // multiple of 512 (groups come in pairs; a CTA's scales load in blocks of
@@ -20,7 +34,8 @@ struct LdPlan {
 // activations, their group sums, the CTA's scales and zeros and the per-warp
 // partial sums of its tiles in shared memory, next to the per-warp rings of
 // codes.
-bool plan_ld(int M, int N, int K, int bits, int group, const DeviceInfo& dev, LdPlan* plan) {
+bool plan_ld(int M, int N, int K, int bits, int group, const DeviceInfo& dev, LdPlan* plan,
+             int variant) {
   using namespace wq::ld;
   if (bits != 4 || group != kGroup || M < 1 || M > kMaxM || N < 1 || K < 4 * kGroup ||
       K % (4 * kGroup) != 0)
@@ -41,13 +56,23 @@ bool plan_ld(int M, int N, int K, int bits, int group, const DeviceInfo& dev, Ld
   p.off_part = uint32_t(round_up(p.off_sz + max_rows * (p.ngroups + 1) * 8, 16));
   p.off_ring =
       uint32_t(round_up(p.off_part + max_tiles * kWarps * kTileRows * size_t(M) * 4, 128));
-  plan->smem = p.off_ring + size_t(kWarps) * kDepth * 1024;
-  return plan->smem <= size_t(dev.max_smem_optin);
+  if (variant < 0 || variant >= kNumLdVariants) return false;
+  const LdVariant v = kLdVariants[variant];
+  plan->variant = variant;
+  plan->smem = p.off_ring + size_t(kWarps) * v.depth * 1024;
+  p.mul_shr4 = 1u << 28;
+  p.mul_shr8 = 1u << 24;
+  p.mul_shr12 = 1u << 20;
+  // CTAs of two launches share an SM only if each takes at most half of it
+  // (1 KB of every CTA's shared memory is reserved by the hardware)
+  const size_t limit = v.min_blocks == 2 ? size_t(dev.max_smem_optin) / 2 - 1024
+                                         : size_t(dev.max_smem_optin);
+  return plan->smem <= limit;
 }
 
-template <bool SYM, int MT>
+template <bool SYM, int MT, int DEPTH, bool FMA_SHIFT, int MINB>
 cudaError_t launch_ld(LdPlan* plan, const DeviceInfo& dev, cudaStream_t s, bool pdl) {
-  auto kernel = &wq::ld::gemv_ld_kernel<SYM, MT>;
+  auto kernel = &wq::ld::gemv_ld_kernel<SYM, MT, DEPTH, FMA_SHIFT, MINB>;
   static int configured[kMaxDevices] = {};
   cudaError_t e = configure_smem(kernel, configured, size_t(dev.max_smem_optin));
   if (e != cudaSuccess) return e;
@@ -67,19 +92,33 @@ cudaError_t launch_ld(LdPlan* plan, const DeviceInfo& dev, cudaStream_t s, bool 
   return cudaLaunchKernelEx(&cfg, kernel, plan->p);
 }
 
+template <bool SYM, int MT>
+cudaError_t launch_ld_v(LdPlan* plan, const DeviceInfo& dev, cudaStream_t s, bool pdl) {
+  switch (plan->variant) {
+    case 1: return launch_ld<SYM, MT, 3, true, 1>(plan, dev, s, pdl);
+    case 2: return launch_ld<SYM, MT, 4, true, 2>(plan, dev, s, pdl);
+    case 3: return launch_ld<SYM, MT, 6, true, 1>(plan, dev, s, pdl);
+    case 4: return launch_ld<SYM, MT, 4, false, 2>(plan, dev, s, pdl);
+    case 5: return launch_ld<SYM, MT, 6, false, 1>(plan, dev, s, pdl);
+    default: return launch_ld<SYM, MT, 3, false, 1>(plan, dev, s, pdl);
+  }
+}
+
 template <bool SYM>
 cudaError_t launch_ld_m(LdPlan* plan, const DeviceInfo& dev, cudaStream_t s, bool pdl) {
   const int M = plan->p.M;
-  if (M == 1) return launch_ld<SYM, 1>(plan, dev, s, pdl);
-  if (M == 2) return launch_ld<SYM, 2>(plan, dev, s, pdl);
-  return launch_ld<SYM, 4>(plan, dev, s, pdl);
+  if (M == 1) return launch_ld_v<SYM, 1>(plan, dev, s, pdl);
+  if (M == 2) return launch_ld_v<SYM, 2>(plan, dev, s, pdl);
+  return launch_ld_v<SYM, 4>(plan, dev, s, pdl);
 }
 
 }  // namespace
 
 bool run_ld(const MatmulArgs& a, cudaError_t* err) {
   LdPlan lp;
-  if (!plan_ld(a.M, a.N, a.K, a.bits, a.group, a.dev, &lp)) return false;
+  if (!plan_ld(a.M, a.N, a.K, a.bits, a.group, a.dev, &lp, g_ld_variant) &&
+      (g_ld_variant == 0 || !plan_ld(a.M, a.N, a.K, a.bits, a.group, a.dev, &lp, 0)))
+    return false;
   lp.p.X = static_cast<const __nv_bfloat16*>(a.X);
   lp.p.Y = a.Y;
   lp.p.codes = static_cast<const uint8_t*>(a.codes);
@@ -105,13 +144,22 @@ int wq_internal_plan_ld(int M, int N, int K, int bits, int group, int sms, int s
   dev.sms = sms;
   dev.max_smem_optin = smem_optin;
   wqh::LdPlan plan;
-  if (!wqh::plan_ld(M, N, K, bits, group, dev, &plan)) return 0;
+  if (!wqh::plan_ld(M, N, K, bits, group, dev, &plan, 0)) return 0;
   const wq::ld::Params& p = plan.p;
   const int64_t v[] = {p.M,      p.N,      p.K,        p.ngroups, p.tiles,
                        p.xs_row_bytes, p.off_sx, p.off_sz, p.off_part, p.off_ring,
                        int64_t(plan.smem), plan.grid};
   for (size_t i = 0; i < sizeof(v) / sizeof(v[0]); ++i) out[i] = v[i];
   return 1;
+}
+
+// Tuning hook, not part of the public ABI: the build variant of the
+// direct-load kernel used by the next calls (0 .. 5; see kLdVariants; a
+// variant that does not fit a shape falls back to 0).  Returns the number
+// of variants.
+int wq_internal_set_ld_variant(int variant) {
+  if (variant >= 0 && variant < wqh::kNumLdVariants) wqh::g_ld_variant = variant;
+  return wqh::kNumLdVariants;
 }
 
 }  // extern "C"

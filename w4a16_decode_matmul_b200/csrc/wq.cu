@@ -40,6 +40,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }  // namespace
 
 int g_kernel_choice = 0;
+int g_prefill_choice = 1;
 
 bool device_info(DeviceInfo* out) {
   int dev = 0;
@@ -207,6 +208,9 @@ wq_status wq_matmul(const void* X, int64_t M, const void* codes, const void* sca
 
   if (M > 32) {
     // prefill: tensor-core GEMM on exact integer weights, binary32 group scaling
+    const int pc = wqh::g_prefill_choice;
+    if (pc != 1 && wqh::run_gemm2(a, &e)) return from_cuda(e);
+    if (pc == 2) return WQ_ERR_UNSUPPORTED;
     if (!wqh::run_gemm(a, &e)) return WQ_ERR_UNSUPPORTED;
     return from_cuda(e);
   }
@@ -346,6 +350,12 @@ const char* wq_internal_last_cuda_error(void) { return cudaGetErrorName(g_last_c
 // CTAs whenever a workspace is given, 4 forces the direct-load kernel (2, 3
 // and 4 return WQ_ERR_UNSUPPORTED where the forced kernel does not apply).
 void wq_internal_set_kernel(int choice) { wqh::g_kernel_choice = choice; }
+
+// Tuning and test hook, not part of the public ABI: the prefill kernel at
+// M > 32 (0 chooses, 1 forces the kernel with both operands in shared
+// memory, 2 forces the kernel with the weights in tensor memory; a forced
+// kernel that does not apply returns WQ_ERR_UNSUPPORTED).
+void wq_internal_set_prefill(int choice) { wqh::g_prefill_choice = choice; }
 
 // Test hook, not part of the public ABI: the number of non-zero flag words
 // in the no-allocation scratch block of the current device (0 when every
