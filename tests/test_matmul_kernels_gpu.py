@@ -2,7 +2,8 @@
 same seeded inputs against the oracle: the balanced kernel with and without
 its workspace (row tiles summed across CTAs, or whole tiles per SM), under
 programmatic dependent launch, the cluster-split kernel it replaces for
-M <= 8, and the direct-load kernel (4-bit codes, groups of 128, M <= 4).  Tolerance as in test_matmul_gpu: |y - y_ref| <= 1e-4 sum|x w|
+M <= 8, the direct-load kernel (4-bit codes, groups of 128, M <= 4) and the
+bulk-staged kernel (the same formats, K a multiple of 1,024).  Tolerance as in test_matmul_gpu: |y - y_ref| <= 1e-4 sum|x w|
 (+ one bfloat16 ulp for bfloat16 out)."""
 import contextlib
 import ctypes
@@ -17,7 +18,7 @@ from tests.gpu_util import check_tolerance, host_bits, oracle_quantize, weight, 
 
 pytestmark = pytest.mark.gpu
 
-AUTO, CLUSTER, BALANCED, BALANCED_SPLIT, DIRECT = 0, 1, 2, 3, 4
+AUTO, CLUSTER, BALANCED, BALANCED_SPLIT, DIRECT, BULK = 0, 1, 2, 3, 4, 5
 
 
 @contextlib.contextmanager
@@ -47,7 +48,7 @@ def workspace_clear():
 
 
 SHAPES = [(1, 14336, 4096), (2, 1000, 4096), (3, 4096, 4096), (5, 1024, 4096), (8, 700, 4096),
-          (1, 4096, 14336), (2, 520, 14336), (1, 77, 1024)]
+          (1, 4096, 14336), (2, 520, 14336), (1, 77, 1024), (4, 300, 2048), (1, 1201, 8192)]
 FORMATS = [(4, 128, False), (4, 128, True), (4, 64, True), (4, 32, False), (8, 128, False), (8, 64, True),
            (8, 32, False)]
 
@@ -90,6 +91,12 @@ def test_balanced_kernel_modes(M, N, K, bits, group, sym):
             outs["direct"] = wq().matmul(Xd, qw)
             outs["direct_pdl"] = wq().matmul(Xd, qw, static_weights=True)
             outs["direct_bf16"] = wq().matmul(Xd, qw, out_dtype=torch.bfloat16)
+    bulk = bits == 4 and group == 128 and M <= 4 and K % 1024 == 0
+    if bulk:
+        with kernel(BULK):
+            outs["bulk"] = wq().matmul(Xd, qw)
+            outs["bulk_pdl"] = wq().matmul(Xd, qw, static_weights=True)
+            outs["bulk_bf16"] = wq().matmul(Xd, qw, out_dtype=torch.bfloat16)
     outs["auto"] = wq().matmul(Xd, qw, static_weights=True)
     torch.cuda.synchronize()
     assert wq().get_device_error() == 0
@@ -102,9 +109,12 @@ def test_balanced_kernel_modes(M, N, K, bits, group, sym):
     assert torch.equal(outs["cluster"], outs["cluster_pdl"])
     if direct:
         assert torch.equal(outs["direct"], outs["direct_pdl"])
+    if bulk:
+        assert torch.equal(outs["bulk"], outs["bulk_pdl"])
 
 
-def test_back_to_back_static_weights():
+@pytest.mark.parametrize("choice", [AUTO, BULK])
+def test_back_to_back_static_weights(choice):
     """A chain of launches with programmatic dependent launch, each over a
     different copy of the weights and reading the previous call's output as
     its activations (so every launch depends on the one before)."""
@@ -114,22 +124,24 @@ def test_back_to_back_static_weights():
     qws = [wq().quantize(W.cuda() * (1.0 + 0.25 * i)) for i in range(3)]
     x = X.cuda()
     chain = [x]
-    for i in range(9):
-        y = wq().matmul(chain[-1], qws[i % 3], static_weights=True)
-        chain.append((y / y.abs().amax()).to(torch.bfloat16))  # keep the scale sane
-    torch.cuda.synchronize()
-    ref = [x]
-    for i in range(9):
-        y = wq().matmul(ref[-1], qws[i % 3])
+    with kernel(choice):
+        for i in range(9):
+            y = wq().matmul(chain[-1], qws[i % 3], static_weights=True)
+            chain.append((y / y.abs().amax()).to(torch.bfloat16))  # keep the scale sane
         torch.cuda.synchronize()
-        ref.append((y / y.abs().amax()).to(torch.bfloat16))
+        ref = [x]
+        for i in range(9):
+            y = wq().matmul(ref[-1], qws[i % 3])
+            torch.cuda.synchronize()
+            ref.append((y / y.abs().amax()).to(torch.bfloat16))
     for a, b in zip(chain, ref):
         assert torch.equal(a, b)
     assert wq().get_device_error() == 0
     assert workspace_clear()
 
 
-def test_graph_replay_with_static_weights():
+@pytest.mark.parametrize("choice", [AUTO, BULK])
+def test_graph_replay_with_static_weights(choice):
     """Captured in a CUDA graph (the bench's launch mode), replayed twice."""
     N, K = 14336, 4096
     W = weight(N, K, seed=0)
@@ -138,7 +150,7 @@ def test_graph_replay_with_static_weights():
     ref = [wq().matmul(X, q) for q in qws]
     s = torch.cuda.Stream()
     Y = torch.empty(1, N, device="cuda")
-    with torch.cuda.stream(s):
+    with kernel(choice), torch.cuda.stream(s):
         wq().matmul(X, qws[0], out=Y, static_weights=True)
         s.synchronize()
         g = torch.cuda.CUDAGraph()
@@ -174,7 +186,8 @@ def test_activation_rows_of_wide_dynamic_range(bits, group, sym):
     torch.cuda.synchronize()
     check_tolerance(Y.cpu().numpy(), y_ref, y_abs, False)
     if bits == 4 and group == 128:
-        with kernel(DIRECT):
-            Y = wq().matmul(X.cuda(), qw)
-        torch.cuda.synchronize()
-        check_tolerance(Y.cpu().numpy(), y_ref, y_abs, False)
+        for choice in (DIRECT, BULK):
+            with kernel(choice):
+                Y = wq().matmul(X.cuda(), qw)
+            torch.cuda.synchronize()
+            check_tolerance(Y.cpu().numpy(), y_ref, y_abs, False)

@@ -62,15 +62,14 @@ constexpr int kBK = 64;      // k per load stage
 constexpr int kMaxLoadStages = 8;
 constexpr int kAStages = 8;  // 32-column A stages in tensor memory
 constexpr int kDequantWarp0 = 2;
-constexpr int kNumEpilogueWarps = 8;
-// threads of a CTA with DW dequantize warps: producer, MMA, dequantize, epilogue
-constexpr int threads_for(int dw) { return (2 + dw + kNumEpilogueWarps) * 32; }
+// threads of a CTA with DW dequantize and EW epilogue warps (and the
+// producer and MMA warps)
+constexpr int threads_for(int dw, int ew) { return (2 + dw + ew) * 32; }
 constexpr int kXStageBytes = kBT * kBK * 2;                          // 16 KB
 constexpr int kTmemCols = 512;
 constexpr int kDCols = kBT;                       // one group accumulator
 constexpr int kACol0 = 2 * kDCols;                // A stages after the two accumulators
 constexpr int kAStageCols = kBK / 2;              // 64 k of bfloat16 pairs
-constexpr int kEpiCols = kBT / 2;                 // tokens per epilogue thread
 
 // mbarrier slots (8 bytes each) in the first KB of shared memory
 constexpr int kBarFull = 0;                    // [kMaxLoadStages] X + codes landed (tx)
@@ -192,15 +191,18 @@ __device__ __forceinline__ void dq8(uint32_t w, float z, uint32_t* o) {
 // LS: load stages in the shared-memory ring; DW: dequantize warps (4: one
 // per tensor-memory lane quarter, a whole stage each; 8: two per quarter,
 // half of a stage's k each).
-template <int BITS, bool SYM, int G, int LS, int DW>
-__global__ void __launch_bounds__(threads_for(DW), 1)
+template <int BITS, bool SYM, int G, int LS, int DW, int EW>
+__global__ void __launch_bounds__(threads_for(DW, EW), 1)
     gemm2_kernel(const __grid_constant__ CUtensorMap tm_x,
                  const __grid_constant__ CUtensorMap tm_codes, const Params p) {
   static_assert(G == 32 || G == 64 || G == 128, "group");
-  static_assert(LS >= 2 && LS <= kMaxLoadStages && (DW == 4 || DW == 8), "roles");
+  static_assert(LS >= 2 && LS <= kMaxLoadStages && (DW == 4 || DW == 8) &&
+                    (EW == 8 || EW == 16), "roles");
   constexpr int kLoadStages = LS;
   constexpr int kNumDequantWarps = DW;
   constexpr int kEpilogueWarp0 = kDequantWarp0 + DW;
+  constexpr int kNumEpilogueWarps = EW;
+  constexpr int kEpiCols = kBT / (EW / 4);         // tokens per epilogue thread: 64 | 32
   constexpr int kStepsPerGroup = G / 16;        // 16-k MMA steps per group
   constexpr int kCodesRowBytes = kBK * BITS / 8;  // 32 | 64 bytes of a row per stage
   constexpr int kChunks = kCodesRowBytes / 16;     // 2 | 4 chunks of 16 bytes
@@ -410,9 +412,9 @@ __global__ void __launch_bounds__(threads_for(DW), 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int e = warp - kEpilogueWarp0;  // 0..7
+    const int e = warp - kEpilogueWarp0;  // 0 .. EW-1
     const int quarter = warp & 3;         // TMEM lanes 32 * quarter ..
-    const int half = e >> 2;              // tokens 64 * half .. of the tile
+    const int half = e >> 2;              // tokens kEpiCols * half .. of the tile
     const int r = 32 * quarter + lane;    // row of the W tile
     const uint32_t lanes = uint32_t(32 * quarter) << 16;
     int gcount = 0;
@@ -435,13 +437,22 @@ __global__ void __launch_bounds__(threads_for(DW), 1)
         }
         tc_fence_after();
         const uint32_t taddr = tmem_base + lanes + uint32_t(db * kDCols + half * kEpiCols);
-        float dv[16];
-#pragma unroll
-        for (int h = 0; h < kEpiCols / 16; ++h) {
-          tmem_ld16(taddr + 16 * h, dv);
+        if constexpr (kEpiCols == 32) {
+          // one load and one wait per group
+          float dv[32];
+          tmem_ld32(taddr, dv);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) S[16 * h + j] = fmaf(sg, dv[j], S[16 * h + j]);
+          for (int j = 0; j < 32; ++j) S[j] = fmaf(sg, dv[j], S[j]);
+        } else {
+          float dv[16];
+#pragma unroll
+          for (int h = 0; h < kEpiCols / 16; ++h) {
+            tmem_ld16(taddr + 16 * h, dv);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) S[16 * h + j] = fmaf(sg, dv[j], S[16 * h + j]);
+          }
         }
         // D_g is read: the MMA warp may overwrite this buffer
         tc_fence_before();

@@ -18,9 +18,10 @@ struct Gemm2Plan {
 // Build variants (load stages, dequantize warps), chosen through an internal
 // tuning hook.
 struct Gemm2Variant {
-  int load_stages, dequant_warps;
+  int load_stages, dequant_warps, epilogue_warps;
 };
-constexpr Gemm2Variant kGemm2Variants[] = {{4, 4}, {8, 4}, {8, 8}, {6, 8}};
+constexpr Gemm2Variant kGemm2Variants[] = {{4, 4, 8},  {8, 4, 8},  {8, 8, 8},
+                                           {6, 4, 16}, {8, 4, 16}, {4, 4, 16}};
 constexpr int kNumGemm2Variants = int(sizeof(kGemm2Variants) / sizeof(kGemm2Variants[0]));
 int g_gemm2_variant = 0;
 
@@ -54,11 +55,11 @@ bool plan_gemm2(int M, int N, int K, int bits, int group, const DeviceInfo& dev,
   return true;
 }
 
-template <int BITS, bool SYM, int G, int LS, int DW>
+template <int BITS, bool SYM, int G, int LS, int DW, int EW>
 cudaError_t launch_gemm2(Gemm2Plan* plan, const DeviceInfo* dev, const void* X, const void* c,
                          cudaStream_t s) {
   using namespace wq::gemm2;
-  auto kernel = &gemm2_kernel<BITS, SYM, G, LS, DW>;
+  auto kernel = &gemm2_kernel<BITS, SYM, G, LS, DW, EW>;
   static int configured[kMaxDevices] = {};
   {
     const cudaError_t e = configure_smem(kernel, configured, size_t(dev->max_smem_optin));
@@ -80,7 +81,7 @@ cudaError_t launch_gemm2(Gemm2Plan* plan, const DeviceInfo* dev, const void* X, 
                     BITS == 4 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
     return cudaErrorInvalidValue;
-  kernel<<<plan->grid, threads_for(DW), plan->smem, s>>>(tx, tc, p);
+  kernel<<<plan->grid, threads_for(DW, EW), plan->smem, s>>>(tx, tc, p);
   return cudaGetLastError();
 }
 
@@ -89,10 +90,12 @@ struct Gemm2Op {
   static cudaError_t run(Gemm2Plan* plan, const DeviceInfo* dev, const void* X, const void* c,
                          cudaStream_t s) {
     switch (plan->variant) {
-      case 1: return launch_gemm2<BITS, SYM, G, 8, 4>(plan, dev, X, c, s);
-      case 2: return launch_gemm2<BITS, SYM, G, 8, 8>(plan, dev, X, c, s);
-      case 3: return launch_gemm2<BITS, SYM, G, 6, 8>(plan, dev, X, c, s);
-      default: return launch_gemm2<BITS, SYM, G, 4, 4>(plan, dev, X, c, s);
+      case 1: return launch_gemm2<BITS, SYM, G, 8, 4, 8>(plan, dev, X, c, s);
+      case 2: return launch_gemm2<BITS, SYM, G, 8, 8, 8>(plan, dev, X, c, s);
+      case 3: return launch_gemm2<BITS, SYM, G, 6, 4, 16>(plan, dev, X, c, s);
+      case 4: return launch_gemm2<BITS, SYM, G, 8, 4, 16>(plan, dev, X, c, s);
+      case 5: return launch_gemm2<BITS, SYM, G, 4, 4, 16>(plan, dev, X, c, s);
+      default: return launch_gemm2<BITS, SYM, G, 4, 4, 8>(plan, dev, X, c, s);
     }
   }
 };
@@ -138,7 +141,7 @@ int wq_internal_plan_gemm2(int M, int N, int K, int bits, int group, int sms, in
 }
 
 // Tuning hook, not part of the public ABI: the build variant of the prefill
-// kernel with the weights in tensor memory (0 .. 3, see kGemm2Variants; one
+// kernel with the weights in tensor memory (0 .. 5, see kGemm2Variants; one
 // that does not fit falls back to 0).  Returns the number of variants.
 int wq_internal_set_gemm2_variant(int variant) {
   if (variant >= 0 && variant < wqh::kNumGemm2Variants) wqh::g_gemm2_variant = variant;

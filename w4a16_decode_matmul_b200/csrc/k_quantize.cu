@@ -4,6 +4,7 @@
 
 #include "host.h"
 #include "quantize.cuh"
+#include "quantize2.cuh"
 
 namespace wqh {
 namespace {
@@ -14,13 +15,27 @@ unsigned grid_for_elements(int64_t total, int sms) {
   return unsigned(std::max<int64_t>(1, std::min<int64_t>(blocks, int64_t(sms) * 16)));
 }
 
+// 0: quantize2_kernel (prefetching, magic-number rounding); 1: the first
+// quantize kernel.  Tuning hook.
+int g_quantize_variant = 0;
+
 template <int B, bool S, int G>
 struct QuantizeOp {
   static cudaError_t run(const void* W, int64_t total, void* c, void* sc, void* z,
                          cudaStream_t s, int sms) {
-    wq::quantize_kernel<B, S, G><<<grid_for_elements(total, sms), 256, 0, s>>>(
-        static_cast<const __half*>(W), total, static_cast<uint8_t*>(c),
-        static_cast<__half*>(sc), static_cast<__half*>(z));
+    if (g_quantize_variant == 1) {
+      wq::quantize_kernel<B, S, G><<<grid_for_elements(total, sms), 256, 0, s>>>(
+          static_cast<const __half*>(W), total, static_cast<uint8_t*>(c),
+          static_cast<__half*>(sc), static_cast<__half*>(z));
+    } else {
+      // one warp per 1,024 weights at a time; four CTAs of 8 warps per SM
+      const int64_t chunks = (total + 1023) / 1024;
+      const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((chunks + 7) / 8,
+                                                                  int64_t(sms) * 4));
+      wq::quantize2_kernel<B, S, G><<<unsigned(blocks), 256, 0, s>>>(
+          static_cast<const __half*>(W), total, static_cast<uint8_t*>(c),
+          static_cast<__half*>(sc), static_cast<__half*>(z));
+    }
     return cudaGetLastError();
   }
 };
@@ -51,3 +66,11 @@ cudaError_t run_dequantize(int bits, bool sym, int group, const void* codes, con
 }
 
 }  // namespace wqh
+
+extern "C" {
+
+// Tuning hook, not part of the public ABI: 0 quantizes with quantize2_kernel
+// (the default), 1 with the first quantize kernel.
+void wq_internal_set_quantize_variant(int variant) { wqh::g_quantize_variant = variant; }
+
+}  // extern "C"
