@@ -2,8 +2,9 @@
 same seeded inputs against the oracle: the balanced kernel with and without
 its workspace (row tiles summed across CTAs, or whole tiles per SM), under
 programmatic dependent launch, the cluster-split kernel it replaces for
-M <= 8, the direct-load kernel (4-bit codes, groups of 128, M <= 4) and the
-bulk-staged kernel (the same formats, K a multiple of 1,024).  Tolerance as in test_matmul_gpu: |y - y_ref| <= 1e-4 sum|x w|
+M <= 8, the direct-load kernel (4-bit codes, groups of 128, M <= 4), the
+bulk-staged kernel (the same formats, K a multiple of 1,024) and the
+k-sliced direct-load kernel (the same formats, K = 4096).  Tolerance as in test_matmul_gpu: |y - y_ref| <= 1e-4 sum|x w|
 (+ one bfloat16 ulp for bfloat16 out)."""
 import contextlib
 import ctypes
@@ -18,7 +19,7 @@ from tests.gpu_util import check_tolerance, host_bits, oracle_quantize, weight, 
 
 pytestmark = pytest.mark.gpu
 
-AUTO, CLUSTER, BALANCED, BALANCED_SPLIT, DIRECT, BULK = 0, 1, 2, 3, 4, 5
+AUTO, CLUSTER, BALANCED, BALANCED_SPLIT, DIRECT, BULK, KSLICE = 0, 1, 2, 3, 4, 5, 6
 
 
 @contextlib.contextmanager
@@ -48,7 +49,8 @@ def workspace_clear():
 
 
 SHAPES = [(1, 14336, 4096), (2, 1000, 4096), (3, 4096, 4096), (5, 1024, 4096), (8, 700, 4096),
-          (1, 4096, 14336), (2, 520, 14336), (1, 77, 1024), (4, 300, 2048), (1, 1201, 8192)]
+          (1, 4096, 14336), (2, 520, 14336), (1, 77, 1024), (4, 300, 2048), (1, 1201, 8192),
+          (4, 1203, 4096), (1, 5, 4096)]
 FORMATS = [(4, 128, False), (4, 128, True), (4, 64, True), (4, 32, False), (8, 128, False), (8, 64, True),
            (8, 32, False)]
 
@@ -97,6 +99,12 @@ def test_balanced_kernel_modes(M, N, K, bits, group, sym):
             outs["bulk"] = wq().matmul(Xd, qw)
             outs["bulk_pdl"] = wq().matmul(Xd, qw, static_weights=True)
             outs["bulk_bf16"] = wq().matmul(Xd, qw, out_dtype=torch.bfloat16)
+    kslice = bits == 4 and group == 128 and M <= 4 and K == 4096
+    if kslice:
+        with kernel(KSLICE):
+            outs["kslice"] = wq().matmul(Xd, qw)
+            outs["kslice_pdl"] = wq().matmul(Xd, qw, static_weights=True)
+            outs["kslice_bf16"] = wq().matmul(Xd, qw, out_dtype=torch.bfloat16)
     outs["auto"] = wq().matmul(Xd, qw, static_weights=True)
     torch.cuda.synchronize()
     assert wq().get_device_error() == 0
@@ -111,9 +119,11 @@ def test_balanced_kernel_modes(M, N, K, bits, group, sym):
         assert torch.equal(outs["direct"], outs["direct_pdl"])
     if bulk:
         assert torch.equal(outs["bulk"], outs["bulk_pdl"])
+    if kslice:
+        assert torch.equal(outs["kslice"], outs["kslice_pdl"])
 
 
-@pytest.mark.parametrize("choice", [AUTO, BULK])
+@pytest.mark.parametrize("choice", [AUTO, BULK, KSLICE])
 def test_back_to_back_static_weights(choice):
     """A chain of launches with programmatic dependent launch, each over a
     different copy of the weights and reading the previous call's output as
@@ -140,14 +150,15 @@ def test_back_to_back_static_weights(choice):
     assert workspace_clear()
 
 
-@pytest.mark.parametrize("choice", [AUTO, BULK])
+@pytest.mark.parametrize("choice", [AUTO, BULK, KSLICE])
 def test_graph_replay_with_static_weights(choice):
     """Captured in a CUDA graph (the bench's launch mode), replayed twice."""
     N, K = 14336, 4096
     W = weight(N, K, seed=0)
     qws = [wq().quantize(W.cuda()) for _ in range(2)]
     X = synth.activation(1, K, seed=1).cuda()
-    ref = [wq().matmul(X, q) for q in qws]
+    with kernel(choice):
+        ref = [wq().matmul(X, q) for q in qws]
     s = torch.cuda.Stream()
     Y = torch.empty(1, N, device="cuda")
     with kernel(choice), torch.cuda.stream(s):
@@ -186,7 +197,7 @@ def test_activation_rows_of_wide_dynamic_range(bits, group, sym):
     torch.cuda.synchronize()
     check_tolerance(Y.cpu().numpy(), y_ref, y_abs, False)
     if bits == 4 and group == 128:
-        for choice in (DIRECT, BULK):
+        for choice in (DIRECT, BULK, KSLICE):
             with kernel(choice):
                 Y = wq().matmul(X.cuda(), qw)
             torch.cuda.synchronize()

@@ -14,8 +14,8 @@ LIB = os.path.join(ROOT, "w4a16_decode_matmul_b200", "libwq.so")
 FIELDS = ["M", "N", "K", "ngroups", "tiles_t", "tiles_w", "num_tiles", "codes_stage_bytes",
           "smem", "grid"]
 SMEM_OPTIN, SMS = 232448, 148
-BW = BT = 128
-BK, STAGES, HEAD = 64, 4, 1024
+BW = 128
+BK, HEAD = 64, 1024
 
 
 @pytest.fixture(scope="module")
@@ -35,7 +35,7 @@ def plan(lib, M, N, K, bits, group):
 
 
 CASES = [(M, N, K, bits, group)
-         for M in (33, 129, 512, 2048, 8192)
+         for M in (33, 64, 65, 129, 512, 2048, 8192)
          for (N, K) in ((14336, 4096), (4096, 14336), (300, 1024), (257, 384))
          for bits in (4, 8) for group in (32, 64, 128) if K % group == 0]
 
@@ -44,6 +44,8 @@ CASES = [(M, N, K, bits, group)
 def test_plan_gemm2(lib, M, N, K, bits, group):
     p = plan(lib, M, N, K, bits, group)
     assert p is not None
+    # 64-token tiles (6 load stages) up to M = 64, 128-token tiles above
+    BT, STAGES = (64, 6) if M <= 64 else (128, 4)
     assert p["ngroups"] == K // group
     assert p["tiles_t"] == -(-M // BT) and p["tiles_w"] == -(-N // BW)
     assert p["num_tiles"] == p["tiles_t"] * p["tiles_w"]
@@ -53,12 +55,16 @@ def test_plan_gemm2(lib, M, N, K, bits, group):
     row = BK * bits // 8
     assert row % 16 == 0 and row in (32, 64)
     assert p["codes_stage_bytes"] == BW * row and p["codes_stage_bytes"] % 1024 == 0
-    # activation boxes: 64 k x 128 tokens of bfloat16 = 16 KB, 128-byte rows
+    # activation boxes: 64 k x BT tokens of bfloat16, 128-byte rows
     x_stage = BT * BK * 2
     assert x_stage % 1024 == 0
     off_codes = HEAD + STAGES * x_stage
     assert off_codes % 1024 == 0
-    assert p["smem"] == off_codes + STAGES * p["codes_stage_bytes"] <= SMEM_OPTIN
+    # the ring of scale / zero blocks (8 slots of 128 rows x 8 groups x 2
+    # tensors) when K / group is a multiple of 8 (the tensor maps' row pitch)
+    meta = 8 * 2 * 128 * 8 * 2 if (K // group) % 8 == 0 else 0
+    assert (off_codes + STAGES * p["codes_stage_bytes"]) % 128 == 0
+    assert p["smem"] == off_codes + STAGES * p["codes_stage_bytes"] + meta <= SMEM_OPTIN
     # every TMA x coordinate (k * 2 bytes for X, bytes for the codes) stays a
     # multiple of 16 bytes
     assert (BK * 2) % 16 == 0 and row % 16 == 0

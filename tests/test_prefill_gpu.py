@@ -52,7 +52,7 @@ def quantize_both(W, bits, group, sym, key=None):
 @pytest.mark.parametrize("bits,group,sym", [(4, 128, False), (4, 64, True), (8, 128, False),
                                             (8, 64, True), (4, 64, False), (8, 128, True),
                                             (4, 32, False), (8, 32, True), (4, 32, True)])
-@pytest.mark.parametrize("M,N,K", [(33, 130, 1024), (128, 256, 1024), (200, 300, 2048),
+@pytest.mark.parametrize("M,N,K", [(33, 130, 1024), (64, 200, 1024), (128, 256, 1024), (200, 300, 2048),
                                    (300, 1000, 512), (256, 128, 4096), (129, 257, 384)])
 def test_reduced_sizes_full_outputs(kernel, M, N, K, bits, group, sym):
     if K % group:

@@ -57,19 +57,23 @@ using gemm::tmem_wait_ld;
 using gemm::umma_desc_sw128;
 
 constexpr int kBW = 128;     // rows of W per tile (MMA M)
-constexpr int kBT = 128;     // tokens per tile (MMA N)
 constexpr int kBK = 64;      // k per load stage
 constexpr int kMaxLoadStages = 8;
 constexpr int kAStages = 8;  // 32-column A stages in tensor memory
 constexpr int kDequantWarp0 = 2;
 // threads of a CTA with DW dequantize and EW epilogue warps (and the
 // producer and MMA warps)
-constexpr int threads_for(int dw, int ew) { return (2 + dw + ew) * 32; }
-constexpr int kXStageBytes = kBT * kBK * 2;                          // 16 KB
+__host__ __device__ constexpr int threads_for(int dw, int ew) { return (2 + dw + ew) * 32; }
 constexpr int kTmemCols = 512;
-constexpr int kDCols = kBT;                       // one group accumulator
-constexpr int kACol0 = 2 * kDCols;                // A stages after the two accumulators
 constexpr int kAStageCols = kBK / 2;              // 64 k of bfloat16 pairs
+// Bytes of one activation stage (BT tokens x 64 k of bfloat16).
+__host__ __device__ constexpr int x_stage_bytes(int bt) { return bt * kBK * 2; }
+// Instruction descriptor: binary32 accumulator, bfloat16 A and B, both
+// K-major, N = BT tokens, M = 128 rows of W.
+__host__ __device__ constexpr uint32_t instr_desc(int bt) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(bt >> 3) << 17) |
+         (uint32_t(kBW >> 4) << 24);
+}
 
 // mbarrier slots (8 bytes each) in the first KB of shared memory
 constexpr int kBarFull = 0;                    // [kMaxLoadStages] X + codes landed (tx)
@@ -79,6 +83,17 @@ constexpr int kBarAEmpty = 24;                 // [kAStages] A stage read by the
 constexpr int kBarDFull = 32;                  // [2] group accumulator ready
 constexpr int kBarDEmpty = 34;                 // [2] group accumulator read
 constexpr int kBarMmaDone = 36;                // every MMA of the CTA finished
+// Ring of 8-group blocks of scales and zeros.  Eight blocks (64 groups) are
+// more than the producer can run ahead of the epilogue (the load ring, the
+// eight A stages and the two accumulators hold at most 34 groups of k at
+// group 32), so the producer never waits on a block the epilogue still needs
+// for work it has not been given.
+constexpr int kMetaSlots = 8;
+constexpr int kMetaGroups = 8;                 // groups per block (16 bytes of a row)
+constexpr int kBarMetaFull = 38;               // [kMetaSlots] block landed (tx)
+constexpr int kBarMetaEmpty = 46;              // [kMetaSlots] block read by every user
+constexpr int kMetaTensorBytes = kBW * kMetaGroups * 2;  // 2 KB: 128 rows x 8 binary16
+constexpr int kMetaSlotBytes = 2 * kMetaTensorBytes;     // scales, then zeros
 constexpr int kTmemSlot = 512;                 // byte offset of the TMEM base address
 constexpr int kAbortSlot = 516;                // byte offset of the abort flag
 constexpr int kSmemHead = 1024;
@@ -92,18 +107,19 @@ struct Params {
   int tiles_t, tiles_w, num_tiles;
   uint32_t codes_stage_bytes;  // kBW * kBK * bits / 8
   uint32_t off_x, off_codes;   // rings (1024-byte aligned)
+  uint32_t off_meta;           // ring of scale / zero blocks (with MT)
 };
 
 // A in tensor memory (M = 128 lanes, K = 16 as eight 32-bit columns of
 // bfloat16 pairs), B from a shared-memory descriptor.
 __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                          uint32_t accumulate) {
+                                          uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
       :
-      : "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(gemm::kInstrDesc), "r"(accumulate)
+      : "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -191,10 +207,15 @@ __device__ __forceinline__ void dq8(uint32_t w, float z, uint32_t* o) {
 // LS: load stages in the shared-memory ring; DW: dequantize warps (4: one
 // per tensor-memory lane quarter, a whole stage each; 8: two per quarter,
 // half of a stage's k each).
-template <int BITS, bool SYM, int G, int LS, int DW, int EW>
+// MT: scales and zeros arrive by TMA in blocks of 8 groups x 128 rows (K /
+// group a multiple of 8, as the tensor maps' row pitch needs); otherwise the
+// dequantize and epilogue threads read them from global memory directly.
+template <int BITS, bool SYM, int G, int LS, int DW, int EW, int BT, bool MT>
 __global__ void __launch_bounds__(threads_for(DW, EW), 1)
     gemm2_kernel(const __grid_constant__ CUtensorMap tm_x,
-                 const __grid_constant__ CUtensorMap tm_codes, const Params p) {
+                 const __grid_constant__ CUtensorMap tm_codes,
+                 const __grid_constant__ CUtensorMap tm_scales,
+                 const __grid_constant__ CUtensorMap tm_zeros, const Params p) {
   static_assert(G == 32 || G == 64 || G == 128, "group");
   static_assert(LS >= 2 && LS <= kMaxLoadStages && (DW == 4 || DW == 8) &&
                     (EW == 8 || EW == 16), "roles");
@@ -202,7 +223,14 @@ __global__ void __launch_bounds__(threads_for(DW, EW), 1)
   constexpr int kNumDequantWarps = DW;
   constexpr int kEpilogueWarp0 = kDequantWarp0 + DW;
   constexpr int kNumEpilogueWarps = EW;
-  constexpr int kEpiCols = kBT / (EW / 4);         // tokens per epilogue thread: 64 | 32
+  static_assert(BT == 64 || BT == 128, "token tile");
+  constexpr int kBT = BT;
+  constexpr int kXStageBytes = x_stage_bytes(BT);
+  constexpr int kDCols = BT;                       // one group accumulator
+  constexpr int kACol0 = 2 * kDCols;               // A stages after the two accumulators
+  constexpr uint32_t kIdesc = instr_desc(BT);
+  constexpr int kEpiCols = kBT / (EW / 4);         // tokens per epilogue thread
+  constexpr int kStagesPerBlock = kMetaGroups * G / kBK;  // load stages per metadata block
   constexpr int kStepsPerGroup = G / 16;        // 16-k MMA steps per group
   constexpr int kCodesRowBytes = kBK * BITS / 8;  // 32 | 64 bytes of a row per stage
   constexpr int kChunks = kCodesRowBytes / 16;     // 2 | 4 chunks of 16 bytes
@@ -232,6 +260,10 @@ __global__ void __launch_bounds__(threads_for(DW, EW), 1)
       mbar_init(&bars[kBarDEmpty + b], kNumEpilogueWarps);
     }
     mbar_init(&bars[kBarMmaDone], 1);
+    for (int b = 0; b < kMetaSlots; ++b) {
+      mbar_init(&bars[kBarMetaFull + b], 1);
+      mbar_init(&bars[kBarMetaEmpty + b], DW + EW);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -261,12 +293,33 @@ __global__ void __launch_bounds__(threads_for(DW, EW), 1)
     if (lane == 0) {
       prefetch_tensormap(&tm_x);
       prefetch_tensormap(&tm_codes);
+      if (MT) {
+        prefetch_tensormap(&tm_scales);
+        if (!SYM) prefetch_tensormap(&tm_zeros);
+      }
       const uint64_t keep = l2_policy_evict_last();  // both operands are reread by other CTAs
-      int issued = 0;
+      int issued = 0, mb = 0;
       bool stop = false;
       for (int tile = blockIdx.x; tile < p.num_tiles && !stop; tile += gridDim.x) {
         const int t0 = (tile / p.tiles_w) * kBT, w0 = (tile % p.tiles_w) * kBW;
         for (int kb = 0; kb < nkb; ++kb, ++issued) {
+          if (MT && kb % kStagesPerBlock == 0) {
+            // the next 8-group block of scales and zeros, ahead of its stages
+            const int ms = mb % kMetaSlots;
+            if (!wait(kBarMetaEmpty + ms, (uint32_t(mb / kMetaSlots) & 1u) ^ 1u)) {
+              stop = true;
+              break;
+            }
+            uint8_t* dst = smem + p.off_meta + ms * kMetaSlotBytes;
+            mbar_arrive_expect_tx(&bars[kBarMetaFull + ms],
+                                  uint32_t((SYM ? 1 : 2) * kMetaTensorBytes));
+            tma_load_2d(dst, &tm_scales, &bars[kBarMetaFull + ms],
+                        (kb / kStagesPerBlock) * kMetaGroups, w0, keep);
+            if (!SYM)
+              tma_load_2d(dst + kMetaTensorBytes, &tm_zeros, &bars[kBarMetaFull + ms],
+                          (kb / kStagesPerBlock) * kMetaGroups, w0, keep);
+            ++mb;
+          }
           const int s = issued % kLoadStages;
           const uint32_t ph = uint32_t(issued / kLoadStages) & 1u;
           if (!wait(kBarEmpty + s, ph ^ 1u)) {
@@ -283,6 +336,8 @@ __global__ void __launch_bounds__(threads_for(DW, EW), 1)
       // every issued copy lands before the CTA can finish
       for (int j = max(0, issued - kLoadStages); j < issued; ++j)
         mbar_wait(&bars[kBarFull + j % kLoadStages], uint32_t(j / kLoadStages) & 1u);
+      for (int j = max(0, mb - kMetaSlots); j < mb; ++j)
+        mbar_wait(&bars[kBarMetaFull + j % kMetaSlots], uint32_t(j / kMetaSlots) & 1u);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -316,7 +371,7 @@ __global__ void __launch_bounds__(threads_for(DW, EW), 1)
               tc_fence_after();
               d = tmem_base + uint32_t(db * kDCols);
             }
-            tc_mma_ts(d, a_addr + uint32_t(8 * k), xdesc + uint64_t(2 * k),
+            tc_mma_ts(d, a_addr + uint32_t(8 * k), xdesc + uint64_t(2 * k), kIdesc,
                       step_in_group > 0 ? 1u : 0u);
             if (++step_in_group == kStepsPerGroup) {
               tc_commit(&bars[kBarDFull + (gcount & 1)]);
@@ -342,7 +397,7 @@ __global__ void __launch_bounds__(threads_for(DW, EW), 1)
     const int r = 32 * quarter + lane;  // row of the W tile = TMEM lane
     const uint32_t lanes = uint32_t(32 * quarter) << 16;
     const int part = (warp - kDequantWarp0) >> 2;  // which share of the stage's k (DW = 8)
-    int ld = 0;
+    int ld = 0, mb = 0;
     bool stop = false;
     for (int tile = blockIdx.x; tile < p.num_tiles && !stop; tile += gridDim.x) {
       const int w0 = (tile % p.tiles_w) * kBW;
@@ -358,6 +413,19 @@ __global__ void __launch_bounds__(threads_for(DW, EW), 1)
           break;
         }
         tc_fence_after();
+        // with MT: this stage's zero points come from the ring's block
+        const __half* zsm = nullptr;
+        if constexpr (MT && !SYM) {
+          const int ms = mb % kMetaSlots;
+          if (kb % kStagesPerBlock == 0 &&
+              !wait(kBarMetaFull + ms, uint32_t(mb / kMetaSlots) & 1u)) {
+            stop = true;
+            break;
+          }
+          zsm = reinterpret_cast<const __half*>(smem + p.off_meta + ms * kMetaSlotBytes +
+                                                kMetaTensorBytes) +
+                r * kMetaGroups;
+        }
         // the stage's codes of row r, unswizzled: chunk c sits at chunk
         // c ^ key (32-byte swizzle: bit 4 of the address XOR bit 7; 64-byte
         // swizzle: bits 4-5 XOR bits 7-8)
@@ -371,7 +439,12 @@ __global__ void __launch_bounds__(threads_for(DW, EW), 1)
             const uint4 v = *reinterpret_cast<const uint4*>(crow + ((c ^ key) << 4));
             const int k0 = kb * kBK + 32 * c;
             float zf = SYM ? 8.f : 0.f;
-            if (!SYM) zf = row_ok ? __half2float(zrow[k0 / G]) : 0.f;
+            if constexpr (!SYM) {
+              if constexpr (MT)
+                zf = __half2float(zsm[(k0 / G) % kMetaGroups]);
+              else
+                zf = row_ok ? __half2float(zrow[k0 / G]) : 0.f;
+            }
             const __nv_bfloat162 zz = __floats2bfloat162_rn(128.f + zf, 128.f + zf);
             const uint32_t zb2 = *reinterpret_cast<const uint32_t*>(&zz);
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -385,7 +458,12 @@ __global__ void __launch_bounds__(threads_for(DW, EW), 1)
             const uint4 v = *reinterpret_cast<const uint4*>(crow + ((c ^ key) << 4));
             const int k0 = kb * kBK + 16 * c;
             float zf = SYM ? 128.f : 0.f;
-            if (!SYM) zf = row_ok ? __half2float(zrow[k0 / G]) : 0.f;
+            if constexpr (!SYM) {
+              if constexpr (MT)
+                zf = __half2float(zsm[(k0 / G) % kMetaGroups]);
+              else
+                zf = row_ok ? __half2float(zrow[k0 / G]) : 0.f;
+            }
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int j = 0; j < 4; ++j) dq8(w[j], zf, o + 8 * cc + 2 * j);
@@ -395,9 +473,14 @@ __global__ void __launch_bounds__(threads_for(DW, EW), 1)
 #pragma unroll
           for (int i = 0; i < kMyCols; ++i) o[i] = 0u;
         }
-        // the codes of this stage are consumed
+        // the codes of this stage are consumed, and with MT the block of zero
+        // points once its last stage is
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[kBarEmpty + s]);
+        if (MT && (kb % kStagesPerBlock == kStagesPerBlock - 1 || kb == nkb - 1)) {
+          if (lane == 0) mbar_arrive(&bars[kBarMetaEmpty + mb % kMetaSlots]);
+          ++mb;
+        }
         const uint32_t col = uint32_t(kACol0 + as * kAStageCols + part * kMyCols);
         if constexpr (kMyCols == 32) {
           tmem_st32(tmem_base + lanes + col, o);
@@ -417,7 +500,7 @@ __global__ void __launch_bounds__(threads_for(DW, EW), 1)
     const int half = e >> 2;              // tokens kEpiCols * half .. of the tile
     const int r = 32 * quarter + lane;    // row of the W tile
     const uint32_t lanes = uint32_t(32 * quarter) << 16;
-    int gcount = 0;
+    int gcount = 0, mb = 0;
     bool stop = false;
     for (int tile = blockIdx.x; tile < p.num_tiles && !stop; tile += gridDim.x) {
       const int t0 = (tile / p.tiles_w) * kBT, w0 = (tile % p.tiles_w) * kBW;
@@ -429,7 +512,24 @@ __global__ void __launch_bounds__(threads_for(DW, EW), 1)
       for (int j = 0; j < kEpiCols; ++j) S[j] = 0.f;
       int done = 0;
       for (int gi = 0; gi < p.ngroups; ++gi, ++gcount) {
-        const float sg = row_ok ? __half2float(srow[gi]) : 0.f;
+        float sg;
+        if constexpr (MT) {
+          const int ms = mb % kMetaSlots;
+          if (gi % kMetaGroups == 0 && !wait(kBarMetaFull + ms, uint32_t(mb / kMetaSlots) & 1u)) {
+            stop = true;
+            break;
+          }
+          sg = __half2float(reinterpret_cast<const __half*>(smem + p.off_meta +
+                                                            ms * kMetaSlotBytes)[r * kMetaGroups +
+                                                                                 gi % kMetaGroups]);
+          if (gi % kMetaGroups == kMetaGroups - 1 || gi == p.ngroups - 1) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[kBarMetaEmpty + ms]);
+            ++mb;
+          }
+        } else {
+          sg = row_ok ? __half2float(srow[gi]) : 0.f;
+        }
         const int db = gcount & 1;
         if (!wait(kBarDFull + db, uint32_t(gcount >> 1) & 1u)) {
           stop = true;
@@ -437,13 +537,20 @@ __global__ void __launch_bounds__(threads_for(DW, EW), 1)
         }
         tc_fence_after();
         const uint32_t taddr = tmem_base + lanes + uint32_t(db * kDCols + half * kEpiCols);
-        if constexpr (kEpiCols == 32) {
+        if constexpr (kEpiCols <= 32) {
           // one load and one wait per group
           float dv[32];
-          tmem_ld32(taddr, dv);
+          if constexpr (kEpiCols == 32) {
+            tmem_ld32(taddr, dv);
+          } else {
+            float d16[16];
+            tmem_ld16(taddr, d16);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) dv[j] = d16[j];
+          }
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) S[j] = fmaf(sg, dv[j], S[j]);
+          for (int j = 0; j < kEpiCols; ++j) S[j] = fmaf(sg, dv[j], S[j]);
         } else {
           float dv[16];
 #pragma unroll

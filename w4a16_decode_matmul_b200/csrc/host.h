@@ -76,6 +76,7 @@ struct MatmulArgs {
 // kernel's scope, true otherwise with the launch result in *err.
 bool run_ld(const MatmulArgs& a, cudaError_t* err);
 bool run_tb(const MatmulArgs& a, cudaError_t* err);
+bool run_ks(const MatmulArgs& a, cudaError_t* err);
 bool run_sk(const MatmulArgs& a, bool split, cudaError_t* err);
 bool run_gemv(const MatmulArgs& a, cudaError_t* err);
 bool run_gemm(const MatmulArgs& a, cudaError_t* err);
@@ -98,7 +99,7 @@ int sk_workspace_ctas();
 // Kernel choice for wq_matmul (tuning and test hook): 0 chooses, 1 forces
 // the cluster-split kernel, 2 the balanced kernel, 3 the balanced kernel
 // with row tiles split across CTAs, 4 the direct-load kernel, 5 the
-// bulk-staged kernel.
+// bulk-staged kernel, 6 the k-sliced direct-load kernel.
 extern int g_kernel_choice;
 
 // Prefill kernel for wq_matmul at M > 32 (tuning and test hook): 0 chooses

@@ -13,6 +13,8 @@ struct Gemm2Plan {
   int grid = 1;
   size_t smem = 0;
   int variant = 0;
+  int bt = 128;   // tokens per tile: 64 for M <= 64 (the MMA's N), else 128
+  bool meta_tma = false;  // scales / zeros by TMA (K / group a multiple of 8)
 };
 
 // Build variants (load stages, dequantize warps), chosen through an internal
@@ -20,8 +22,7 @@ struct Gemm2Plan {
 struct Gemm2Variant {
   int load_stages, dequant_warps, epilogue_warps;
 };
-constexpr Gemm2Variant kGemm2Variants[] = {{4, 4, 8},  {8, 4, 8},  {8, 8, 8},
-                                           {6, 4, 16}, {8, 4, 16}, {4, 4, 16}};
+constexpr Gemm2Variant kGemm2Variants[] = {{4, 4, 8}, {8, 4, 8}, {6, 4, 16}};
 constexpr int kNumGemm2Variants = int(sizeof(kGemm2Variants) / sizeof(kGemm2Variants[0]));
 int g_gemm2_variant = 0;
 
@@ -31,35 +32,41 @@ bool plan_gemm2(int M, int N, int K, int bits, int group, const DeviceInfo& dev,
   using namespace wq::gemm2;
   if (variant < 0 || variant >= kNumGemm2Variants) return false;
   plan->variant = variant;
-  const int stages = kGemm2Variants[variant].load_stages;
+  // the 64-token tile has one build: 6 load stages, 4 dequantize and 8
+  // epilogue warps
+  const int stages = M <= 64 ? 6 : kGemm2Variants[variant].load_stages;
   if (group != 32 && group != 64 && group != 128) return false;
   if (bits != 4 && bits != 8) return false;
   if (K % kBK != 0 || K % group != 0 || M < 1 || N < 1) return false;
   wq::gemm2::Params& p = plan->p;
   p = wq::gemm2::Params{};
+  plan->bt = M <= 64 ? 64 : 128;
+  const int bt = plan->bt;
   p.M = M;
   p.N = N;
   p.K = K;
   p.ngroups = K / group;
-  p.tiles_t = (M + kBT - 1) / kBT;
+  p.tiles_t = (M + bt - 1) / bt;
   p.tiles_w = (N + kBW - 1) / kBW;
   const long long tiles = (long long)p.tiles_t * p.tiles_w;
   if (tiles > 0x7fffffffLL) return false;
   p.num_tiles = int(tiles);
   p.codes_stage_bytes = uint32_t(kBW * kBK * bits / 8);
   p.off_x = kSmemHead;
-  p.off_codes = p.off_x + uint32_t(stages * kXStageBytes);
-  plan->smem = p.off_codes + size_t(stages) * p.codes_stage_bytes;
+  p.off_codes = p.off_x + uint32_t(stages * x_stage_bytes(bt));
+  p.off_meta = p.off_codes + uint32_t(stages) * p.codes_stage_bytes;
+  plan->meta_tma = p.ngroups % kMetaGroups == 0;
+  plan->smem = p.off_meta + (plan->meta_tma ? size_t(kMetaSlots) * kMetaSlotBytes : 0);
   if (plan->smem > size_t(dev.max_smem_optin)) return false;
   plan->grid = std::min(p.num_tiles, dev.sms);
   return true;
 }
 
-template <int BITS, bool SYM, int G, int LS, int DW, int EW>
+template <int BITS, bool SYM, int G, int LS, int DW, int EW, int BT, bool MT>
 cudaError_t launch_gemm2(Gemm2Plan* plan, const DeviceInfo* dev, const void* X, const void* c,
-                         cudaStream_t s) {
+                         const void* sc, const void* z, cudaStream_t s) {
   using namespace wq::gemm2;
-  auto kernel = &gemm2_kernel<BITS, SYM, G, LS, DW, EW>;
+  auto kernel = &gemm2_kernel<BITS, SYM, G, LS, DW, EW, BT, MT>;
   static int configured[kMaxDevices] = {};
   {
     const cudaError_t e = configure_smem(kernel, configured, size_t(dev->max_smem_optin));
@@ -67,10 +74,10 @@ cudaError_t launch_gemm2(Gemm2Plan* plan, const DeviceInfo* dev, const void* X, 
   }
   const wq::gemm2::Params& p = plan->p;
   CUtensorMap tx, tc;
-  // X [M][K] bfloat16, boxes of 64 k x 128 tokens, 128-byte swizzle (the
+  // X [M][K] bfloat16, boxes of 64 k x BT tokens, 128-byte swizzle (the
   // K-major canonical layout of the MMA's B operand)
   if (!encode_2d_ex(&tx, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, uint64_t(p.K), uint64_t(p.M),
-                    uint32_t(kBK), uint32_t(kBT), CU_TENSOR_MAP_SWIZZLE_128B,
+                    uint32_t(kBK), uint32_t(BT), CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
     return cudaErrorInvalidValue;
   // codes [N][K*bits/8] bytes, boxes of 64 k x 128 rows, swizzled so that
@@ -81,22 +88,39 @@ cudaError_t launch_gemm2(Gemm2Plan* plan, const DeviceInfo* dev, const void* X, 
                     BITS == 4 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
     return cudaErrorInvalidValue;
-  kernel<<<plan->grid, threads_for(DW, EW), plan->smem, s>>>(tx, tc, p);
+  // scales / zeros [N][ngroups] binary16, boxes of 8 groups x 128 rows
+  CUtensorMap ts, tz;
+  std::memcpy(&ts, &tx, sizeof(tx));
+  std::memcpy(&tz, &tx, sizeof(tx));
+  if (MT) {
+    if (!encode_2d(&ts, sc, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, uint64_t(p.ngroups),
+                   uint64_t(p.N), uint32_t(kMetaGroups), uint32_t(kBW)))
+      return cudaErrorInvalidValue;
+    if (!SYM && !encode_2d(&tz, z, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, uint64_t(p.ngroups),
+                           uint64_t(p.N), uint32_t(kMetaGroups), uint32_t(kBW)))
+      return cudaErrorInvalidValue;
+  }
+  kernel<<<plan->grid, threads_for(DW, EW), plan->smem, s>>>(tx, tc, ts, tz, p);
   return cudaGetLastError();
+}
+
+template <int BITS, bool SYM, int G, bool MT>
+cudaError_t launch_gemm2_v(Gemm2Plan* plan, const DeviceInfo* dev, const void* X, const void* c,
+                           const void* sc, const void* z, cudaStream_t s) {
+  if (plan->bt == 64) return launch_gemm2<BITS, SYM, G, 6, 4, 8, 64, MT>(plan, dev, X, c, sc, z, s);
+  switch (plan->variant) {
+    case 1: return launch_gemm2<BITS, SYM, G, 8, 4, 8, 128, MT>(plan, dev, X, c, sc, z, s);
+    case 2: return launch_gemm2<BITS, SYM, G, 6, 4, 16, 128, MT>(plan, dev, X, c, sc, z, s);
+    default: return launch_gemm2<BITS, SYM, G, 4, 4, 8, 128, MT>(plan, dev, X, c, sc, z, s);
+  }
 }
 
 template <int BITS, bool SYM, int G>
 struct Gemm2Op {
   static cudaError_t run(Gemm2Plan* plan, const DeviceInfo* dev, const void* X, const void* c,
-                         cudaStream_t s) {
-    switch (plan->variant) {
-      case 1: return launch_gemm2<BITS, SYM, G, 8, 4, 8>(plan, dev, X, c, s);
-      case 2: return launch_gemm2<BITS, SYM, G, 8, 8, 8>(plan, dev, X, c, s);
-      case 3: return launch_gemm2<BITS, SYM, G, 6, 4, 16>(plan, dev, X, c, s);
-      case 4: return launch_gemm2<BITS, SYM, G, 8, 4, 16>(plan, dev, X, c, s);
-      case 5: return launch_gemm2<BITS, SYM, G, 4, 4, 16>(plan, dev, X, c, s);
-      default: return launch_gemm2<BITS, SYM, G, 4, 4, 8>(plan, dev, X, c, s);
-    }
+                         const void* sc, const void* z, cudaStream_t s) {
+    return plan->meta_tma ? launch_gemm2_v<BITS, SYM, G, true>(plan, dev, X, c, sc, z, s)
+                          : launch_gemm2_v<BITS, SYM, G, false>(plan, dev, X, c, sc, z, s);
   }
 };
 
@@ -113,7 +137,8 @@ bool run_gemm2(const MatmulArgs& a, cudaError_t* err) {
     gp.p.Y_f32 = static_cast<float*>(a.Y);
   gp.p.scales = static_cast<const __half*>(a.scales);
   gp.p.zeros = static_cast<const __half*>(a.zeros);
-  *err = dispatch_format<Gemm2Op>(a.bits, a.sym, a.group, &gp, &a.dev, a.X, a.codes, a.stream);
+  *err = dispatch_format<Gemm2Op>(a.bits, a.sym, a.group, &gp, &a.dev, a.X, a.codes, a.scales,
+                                 a.zeros, a.stream);
   return true;
 }
 
@@ -141,7 +166,7 @@ int wq_internal_plan_gemm2(int M, int N, int K, int bits, int group, int sms, in
 }
 
 // Tuning hook, not part of the public ABI: the build variant of the prefill
-// kernel with the weights in tensor memory (0 .. 5, see kGemm2Variants; one
+// kernel with the weights in tensor memory (0 .. 2, see kGemm2Variants; one
 // that does not fit falls back to 0).  Returns the number of variants.
 int wq_internal_set_gemm2_variant(int variant) {
   if (variant >= 0 && variant < wqh::kNumGemm2Variants) wqh::g_gemm2_variant = variant;
