@@ -352,6 +352,7 @@ def run_wq(args):
     quant = quantize_points(wq, torch, dev, stream)
     model_quant = whole_model_quantize(wq, torch, dev, stream)
     q4k = q4k_point(wq, torch, dev, stream)
+    w8 = w8_gemv_point(wq, torch, dev, stream)
 
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
@@ -382,6 +383,7 @@ def run_wq(args):
         "quantize_layer": quant,
         "quantize_whole_model": model_quant,
         "q4k_gemv": q4k,
+        "w8a16_gemv": w8,
         "page2_h100_bandwidth_model": PAGE2_H100_CONTEXT,
     }
     if world == 1:
@@ -635,9 +637,49 @@ def q4k_point(wq, torch, dev, stream, reps: int = 10):
                    f"graph of {pool_n} launches over rotating copies"}
 
 
+def w8_gemv_point(wq, torch, dev, stream, reps: int = 10):
+    """The same layer with 8-bit codes (W8A16, asymmetric, group 128): the
+    fused M=1 matmul from a CUDA graph over a rotating pool of copies larger
+    than 4x the L2 (programmatic dependent launch); bytes moved and the
+    fraction of the HBM copy peak."""
+    import synth
+    W = synth.weight(N, K, seed=0).to(dev)
+    base = wq.quantize(W, bits=8, group=GROUP, symmetric=False)
+    del W
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    pool_n = max(2, -(-4 * l2 // base.nbytes) + 1)
+    pool = [wq.QuantizedWeight(base.codes.clone(), base.scales.clone(), base.zeros.clone(),
+                               N, K, 8, GROUP, False) for _ in range(pool_n)]
+    X = synth.activation(M, K, seed=1).to(dev)
+    Y = torch.empty(M, N, dtype=torch.float32, device=dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        wq.matmul(X, pool[0], out=Y, static_weights=True)
+        stream.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            for q in pool:
+                wq.matmul(X, q, out=Y, static_weights=True)
+        g.replay()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e.record(stream)
+    torch.cuda.synchronize(dev)
+    us = s.elapsed_time(e) * 1e3 / (pool_n * reps)
+    moved = algorithmic_bytes(bits=8)
+    peak, kind = measured_peaks()
+    return {"us_per_layer": round(us, 3), "gbs": round(moved / us / 1e3, 1),
+            "bytes_per_layer": moved, "frac": round(moved / us / 1e3 / peak, 4),
+            "peak_kind": f"{kind} HBM copy",
+            "how": f"M=1, K={K}, N={N}, 8-bit asymmetric group 128, CUDA graph of {pool_n} "
+                   "launches over rotating copies, programmatic dependent launch"}
+
+
 def prefill_points(wq, torch, dev, reps: int = 8):
-    """The prefill-shaped matmul (M in {512, 2048, 8192}, K=4096, N=14336,
-    INT4 asymmetric group 128) on the tensor cores next to a dense bf16 GEMM
+    """The prefill-shaped matmul (M in {512, 2048, 8192}, and the mid sizes 64
+    and 256; K=4096, N=14336, INT4 asymmetric group 128) on the tensor cores
+    next to a dense bf16 GEMM
     of the same shape (torch/cuBLAS); TFLOP/s = 2 M N K / time, and the
     fraction of the measured dense bf16 peak (burst)."""
     import synth
@@ -645,7 +687,7 @@ def prefill_points(wq, torch, dev, reps: int = 8):
     Wd = torch.randn(N, K, device=dev, dtype=torch.bfloat16)
     peak = measured_bf16_tflops()
     out = {}
-    for m in (512, 2048, 8192):
+    for m in (64, 256, 512, 2048, 8192):
         X = synth.activation(m, K, seed=3).to(dev)
         Y = torch.empty(m, N, device=dev, dtype=torch.float32)
         Yd = torch.empty(m, N, device=dev, dtype=torch.bfloat16)

@@ -82,23 +82,21 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_ks_kernel(const Params p) {
   constexpr size_t kTileStride = size_t(kTileRows) * kRowBytes;
   const uint32_t ring =
       smem_addr(smem) + p.off_ring + uint32_t(warp * DEPTH * 1024 + lane * 16);
-  // full tiles: every row < N; the CTA's last tile may be partial
-  const bool last_partial = tb1 * kTileRows > p.N;
+  // tiles [0, nfull) of the CTA have every row < N; only the last may not
+  const int nfull = tb1 * kTileRows > p.N ? ntiles - 1 : ntiles;
   int fetched = 0;
   auto fetch = [&](int slot) {
-    if (fetched < ntiles) {
-      const uint32_t dst = ring + uint32_t(slot) * 1024;
-      if (!last_partial || fetched < ntiles - 1) {
-        ld::cp_async16(dst, src, true);
-        ld::cp_async16(dst + 512, src + 4 * kRowBytes, true);
-      } else {
-        const int row = (tb0 + fetched) * kTileRows + r;
-        ld::cp_async16(dst, row < p.N ? src : p.codes, row < p.N);
-        ld::cp_async16(dst + 512, row + 4 < p.N ? src + 4 * kRowBytes : p.codes, row + 4 < p.N);
-      }
-      src += kTileStride;
-      ++fetched;
+    const uint32_t dst = ring + uint32_t(slot) * 1024;
+    if (fetched < nfull) {
+      ld::cp_async16(dst, src, true);
+      ld::cp_async16(dst + 512, src + 4 * kRowBytes, true);
+    } else if (fetched < ntiles) {
+      const int row = (tb0 + fetched) * kTileRows + r;
+      ld::cp_async16(dst, row < p.N ? src : p.codes, row < p.N);
+      ld::cp_async16(dst + 512, row + 4 < p.N ? src + 4 * kRowBytes : p.codes, row + 4 < p.N);
     }
+    src += kTileStride;  // never dereferenced past the CTA's last tile
+    ++fetched;
     ld::cp_async_commit();
   };
 
@@ -172,57 +170,66 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_ks_kernel(const Params p) {
   float* dst = part + size_t(warp) * per_tile;
   const size_t part_tile_stride = size_t(kWarps) * per_tile;
   // the partial sums of this warp's slots: every slot of every tile is
-  // written below (rows past N included), so no clearing is needed
+  // written below (rows past N included), so no clearing is needed; the
+  // {s, 128 + z} table was written by all threads
+  __syncthreads();
 
-  for (int it = 0; it < ntiles; ++it) {
-    const int slot = it % DEPTH;
-    ld::cp_async_wait<DEPTH - 1>();
-    const uint32_t a = ring + uint32_t(slot) * 1024;
-    const uint4 c0 = lds128(a);
-    const uint4 c1 = lds128(a + 512);
-    float d[4] = {0.f, 0.f, 0.f, 0.f};
-    const uint32_t w0[4] = {c0.x, c0.y, c0.z, c0.w};
-    const uint32_t w1[4] = {c1.x, c1.y, c1.z, c1.w};
+  // Every lane computes its epilogue values (a lane and its partner L ^ 6
+  // are both owners or both not; only owners' sums are stored), so the loop
+  // has no branch but its end; slots are compile-time constants.
+  const int mrow = MT == 1 ? 1 : p.M;
+  const bool st0 = hh == 0 && use0, st1 = hh == 0 && use1;
+  for (int it0 = 0; it0 < ntiles; it0 += DEPTH) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      uint32_t pa[4], pb[4];
-      unpack_u4(w0[q], pa);
-      unpack_u4(w1[q], pb);
-      const uint32_t a_even[4] = {pa[0], pb[0], pa[1], pb[1]};
-      const uint32_t b_even[2] = {xf[q].x, xf[q].y};
-      const uint32_t a_odd[4] = {pa[2], pb[2], pa[3], pb[3]};
-      const uint32_t b_odd[2] = {xf[q].z, xf[q].w};
-      mma_bf16_16816(d, a_even, b_even);
-      mma_bf16_16816(d, a_odd, b_odd);
-    }
-    // the slot's bytes are used: refill it with the unit DEPTH tiles on
-    fetch(slot);
-    // y += s (C - (128 + z) Sx) for tile rows rr0 and rr0 + 4, in binary32
-    float y[4] = {0.f, 0.f, 0.f, 0.f};
-    if (owner) {
+    for (int slot = 0; slot < DEPTH; ++slot) {
+      if (it0 + slot >= ntiles) break;
+      ld::cp_async_wait<DEPTH - 1>();
+      const uint32_t a = ring + uint32_t(slot) * 1024;
+      const uint4 c0 = lds128(a);
+      const uint4 c1 = lds128(a + 512);
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint32_t w0[4] = {c0.x, c0.y, c0.z, c0.w};
+      const uint32_t w1[4] = {c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t pa[4], pb[4];
+        unpack_u4(w0[q], pa);
+        unpack_u4(w1[q], pb);
+        const uint32_t a_even[4] = {pa[0], pb[0], pa[1], pb[1]};
+        const uint32_t b_even[2] = {xf[q].x, xf[q].y};
+        const uint32_t a_odd[4] = {pa[2], pb[2], pa[3], pb[3]};
+        const uint32_t b_odd[2] = {xf[q].z, xf[q].w};
+        mma_bf16_16816(d, a_even, b_even);
+        mma_bf16_16816(d, a_odd, b_odd);
+      }
+      // the slot's bytes are used: refill it with the unit DEPTH tiles on
+      fetch(slot);
+      // y = s (C - (128 + z) Sx) for tile rows rr0 and rr0 + 4, in binary32;
+      // the row's two groups are then added (lanes L and L ^ 6; binary32
+      // addition commutes, so both lanes hold the same sum)
       const float2 e0 = szp[0];
       const float2 e1 = szp[4 * kSzStride];
-      y[0] = e0.x * fmaf(-e0.y, sx0, d[0]);
-      y[2] = e1.x * fmaf(-e1.y, sx0, d[2]);
-      y[1] = e0.x * fmaf(-e0.y, sx1, d[1]);
-      y[3] = e1.x * fmaf(-e1.y, sx1, d[3]);
+      szp += kTileRows * kSzStride;
+      float y0 = e0.x * fmaf(-e0.y, sx0, d[0]);
+      float y2 = e1.x * fmaf(-e1.y, sx0, d[2]);
+      y0 += __shfl_xor_sync(0xffffffffu, y0, 6);
+      y2 += __shfl_xor_sync(0xffffffffu, y2, 6);
+      if (st0) {
+        dst[rr0 * mrow + m0] = y0;
+        dst[(rr0 + 4) * mrow + m0] = y2;
+      }
+      if constexpr (MT > 1) {
+        float y1 = e0.x * fmaf(-e0.y, sx1, d[1]);
+        float y3 = e1.x * fmaf(-e1.y, sx1, d[3]);
+        y1 += __shfl_xor_sync(0xffffffffu, y1, 6);
+        y3 += __shfl_xor_sync(0xffffffffu, y3, 6);
+        if (st1) {
+          dst[rr0 * mrow + m1] = y1;
+          dst[(rr0 + 4) * mrow + m1] = y3;
+        }
+      }
+      dst += part_tile_stride;
     }
-    szp += kTileRows * kSzStride;
-    // the row's two groups (lanes L and L ^ 6), group A's lane first
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float other = __shfl_xor_sync(0xffffffffu, y[i], 6);
-      y[i] = hh == 0 ? y[i] + other : other + y[i];
-    }
-    if (hh == 0 && use0) {
-      dst[rr0 * p.M + m0] = y[0];
-      dst[(rr0 + 4) * p.M + m0] = y[2];
-    }
-    if (hh == 0 && use1) {
-      dst[rr0 * p.M + m1] = y[1];
-      dst[(rr0 + 4) * p.M + m1] = y[3];
-    }
-    dst += part_tile_stride;
   }
   ld::cp_async_wait<0>();
   __syncthreads();

@@ -15,9 +15,15 @@ struct KsPlan {
   size_t smem = 0;
 };
 
+// 0: one CTA per SM with at most half an SM of shared memory, so that the
+// next launch's CTA can stream on the same SM (ring 3 to 5 units deep);
+// 1: one CTA per SM with the whole SM (ring up to 8 units deep); 2: two
+// CTAs per SM, each with at most half of it.
+int g_ks_mode = 0;
+
 // Scope: 4-bit codes in groups of 128, K = 4096, M <= 4.  One CTA per SM (at
-// most one per 8-row tile), at most half an SM of shared memory; the ring
-// is as deep (3 to 5 units per warp) as that allows.
+// most one per 8-row tile); the ring is as deep as the shared memory of the
+// mode allows.
 bool plan_ks(int M, int N, int K, int bits, int group, const DeviceInfo& dev, KsPlan* plan) {
   using namespace wq::ks;
   if (bits != 4 || group != 128 || K != kK || M < 1 || M > kMaxM || N < 1) return false;
@@ -26,14 +32,16 @@ bool plan_ks(int M, int N, int K, int bits, int group, const DeviceInfo& dev, Ks
   p.M = M;
   p.N = N;
   p.tiles = (N + kTileRows - 1) / kTileRows;
-  plan->grid = std::min(p.tiles, dev.sms);
+  plan->grid = std::min(p.tiles, (g_ks_mode == 2 ? 2 : 1) * dev.sms);
   const size_t max_tiles = size_t((p.tiles + plan->grid - 1) / plan->grid);
   p.off_sz = 0;
   p.off_part = uint32_t(round_up(max_tiles * kTileRows * (kK / 128 + 1) * 8, 16));
   p.off_ring = uint32_t(round_up(p.off_part + max_tiles * kWarps * kTileRows * size_t(M) * 4, 128));
-  const size_t half_sm = size_t(dev.max_smem_optin) / 2 - 1024;
-  int depth = 5;
-  while (depth >= 3 && p.off_ring + size_t(kWarps) * depth * 1024 > half_sm) --depth;
+  const size_t limit = g_ks_mode == 1 ? size_t(dev.max_smem_optin)
+                                       : size_t(dev.max_smem_optin) / 2 - 1024;
+  int depth = g_ks_mode == 1 ? 8 : 5;
+  while (depth >= 3 && p.off_ring + size_t(kWarps) * depth * 1024 > limit) --depth;
+  if (depth == 7) depth = 6;
   if (depth < 3) return false;
   plan->depth = depth;
   plan->smem = p.off_ring + size_t(kWarps) * depth * 1024;
@@ -65,6 +73,8 @@ cudaError_t launch_ks(KsPlan* plan, const DeviceInfo& dev, cudaStream_t s, bool 
 template <bool SYM, int MT>
 cudaError_t launch_ks_d(KsPlan* plan, const DeviceInfo& dev, cudaStream_t s, bool pdl) {
   switch (plan->depth) {
+    case 8: return launch_ks<SYM, MT, 8>(plan, dev, s, pdl);
+    case 6: return launch_ks<SYM, MT, 6>(plan, dev, s, pdl);
     case 5: return launch_ks<SYM, MT, 5>(plan, dev, s, pdl);
     case 4: return launch_ks<SYM, MT, 4>(plan, dev, s, pdl);
     default: return launch_ks<SYM, MT, 3>(plan, dev, s, pdl);
@@ -98,6 +108,11 @@ bool run_ks(const MatmulArgs& a, cudaError_t* err) {
 }  // namespace wqh
 
 extern "C" {
+
+// Tuning hook, not part of the public ABI: the k-sliced kernel's shared
+// memory mode (0: one CTA per SM in half of it, 1: one CTA per SM, the whole
+// SM, 2: two CTAs per SM).
+void wq_internal_set_ks_mode(int mode) { wqh::g_ks_mode = mode >= 0 && mode <= 2 ? mode : 0; }
 
 // Test hook, not part of the public ABI: the k-sliced kernel's plan for a
 // device with `sms` SMs and `smem_optin` bytes of shared memory per block,
