@@ -48,7 +48,7 @@ CSRC = os.path.join(ROOT, "w4a16_decode_matmul_b200", "csrc")
 # What decides the timed kernel: its device code, the host plan and launch of
 # it, and the matmul entry point that chooses it.
 KERNEL_SOURCES = [os.path.join(CSRC, f)
-                  for f in ("gemv_ld.cuh", "unpack.cuh", "common.cuh", "k_ld.cu")]
+                  for f in ("gemv_ks.cuh", "gemv_ld.cuh", "unpack.cuh", "common.cuh", "k_ks.cu")]
 KERNEL_HOST_SECTIONS = [
     ("wq_status wq_matmul(const void* X, int64_t M,",
      "// ------------------------------------------------------ no-allocation entry"),
@@ -74,7 +74,7 @@ def algorithmic_bytes(m: int = M, n: int = N, k: int = K, bits: int = BITS,
 
 def kernel_source_hash() -> str:
     """Hash of the sources that decide the timed kernel (device headers, its
-    plan and launch in k_ld.cu, and the kernel choice in wq.cu)."""
+    plan and launch in k_ks.cu, and the kernel choice in wq.cu)."""
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
         h.update(open(f, "rb").read())

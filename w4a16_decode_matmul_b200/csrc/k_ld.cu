@@ -26,7 +26,7 @@ constexpr LdVariant kLdVariants[] = {
     {3, false, 1}, {3, true, 1}, {4, true, 2}, {6, true, 1}, {4, false, 2}, {6, false, 1},
 };
 constexpr int kNumLdVariants = int(sizeof(kLdVariants) / sizeof(kLdVariants[0]));
-int g_ld_variant = 0;
+int g_ld_variant = 4;  // measured fastest (4-deep ring, two CTAs per SM)
 
 // Plan the direct-load kernel: 4-bit codes in groups of 128 with K a
 // multiple of 512 (groups come in pairs; a CTA's scales load in blocks of

@@ -15,8 +15,8 @@ unsigned grid_for_elements(int64_t total, int sms) {
   return unsigned(std::max<int64_t>(1, std::min<int64_t>(blocks, int64_t(sms) * 16)));
 }
 
-// 0: quantize2_kernel (prefetching, magic-number rounding); 1: the first
-// quantize kernel.  Tuning hook.
+// 0: quantize2_kernel (prefetching, paired binary32 rounding, exact ties
+// fixed per word); 1: the first quantize kernel.  Tuning hook.
 int g_quantize_variant = 0;
 
 template <int B, bool S, int G>
@@ -28,10 +28,10 @@ struct QuantizeOp {
           static_cast<const __half*>(W), total, static_cast<uint8_t*>(c),
           static_cast<__half*>(sc), static_cast<__half*>(z));
     } else {
-      // one warp per 1,024 weights at a time; four CTAs of 8 warps per SM
+      // one warp per 1,024 weights at a time; three CTAs of 8 warps per SM
       const int64_t chunks = (total + 1023) / 1024;
       const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((chunks + 7) / 8,
-                                                                  int64_t(sms) * 4));
+                                                                  int64_t(sms) * 3));
       wq::quantize2_kernel<B, S, G><<<unsigned(blocks), 256, 0, s>>>(
           static_cast<const __half*>(W), total, static_cast<uint8_t*>(c),
           static_cast<__half*>(sc), static_cast<__half*>(z));

@@ -14,19 +14,22 @@
 //     lanes' shuffles;
 //   * forms the binary16 scale (binary64 quotient rounded up twice) and the
 //     zero point exactly as quantize.cuh does;
-//   * rounds t = w * inv, inv = 1/s rounded to nearest (|t - w/s| < 2^-15,
-//     see quantize.cuh), by adding C + z with C = 1.5 * 2^23: the binary32
-//     sum lands on the integer grid, so u - C = rint(t + z) = rint(t) + z for
-//     every t that is not within 2^-12 of a half-integer.  Whether any lane
-//     holds such a t is decided once per chunk (the largest |t - rint(t)|);
-//     if one does, the chunk's codes are recomputed with the exact tie rule
-//     of quantize.cuh (rint_quotient).  The lower clamp of the asymmetric
-//     codes never binds (rint is monotone and rint(lo/s) = -z), the upper one
-//     can (two half-way roundings up); symmetric codes never leave
-//     [-2^(b-1)+1, 2^(b-1)-1] (|w| <= max|w| <= s (2^(b-1)-1));
-//   * packs four codes at a time as the exact binary32 integer
-//     q0 + 16 q1 + 256 q2 + 4096 q3 (or two 8-bit codes q0 + 256 q1), whose
-//     low 16 bits are read off after adding 2^23.
+//   * rounds t = w * inv, inv = 1/s rounded to nearest, with paired binary32
+//     arithmetic: u = t + (C + zoff), C = 1.5 * 2^23, lands on the integer
+//     grid, so the bits of u less those of C are rint(t) + zoff, the stored
+//     code, whose low byte goes straight into the packed word.  |t - w/s| <=
+//     qmax * 2^-23 < 2^-15 (two roundings of relative size 2^-24), so a t
+//     farther than 2^-14 from every half-integer rounds as w/s does.  For
+//     such a t neither clamp can bind either: asymmetric, w/s + z lies in
+//     [-0.5 - 2^-16, qmax + 0.5 + 2^-16] (s >= (hi - lo)/qmax and z is
+//     -lo/s rounded), so leaving [0, qmax] needs w/s + z within 2^-16 of
+//     -0.5 or qmax + 0.5; symmetric, |w/s| <= qmax.  A mask records, per
+//     weight, whether t is that far (e = t - rint(t) is exact, and the sign
+//     of e^2 - (0.5 - 2^-14)^2 is taken in one fused rounding);
+//   * recomputes, only where the mask says so (in practice where w/s is
+//     exactly a half-integer, ~3e-4 of the weights of a normal layer), the
+//     packed word holding the weight with the exact tie rule of quantize.cuh
+//     (rint_quotient) and both clamps, from the weights in global memory.
 #pragma once
 
 #include "common.cuh"
@@ -47,53 +50,73 @@ __device__ __forceinline__ uint32_t pack_codes_f(const float* q) {
   }
 }
 
-template <int BITS>
-struct CodeWords {
-  uint32_t w[BITS];
-};
+// One pair of weights (a binary16 pair) through the fast path with paired
+// binary32 arithmetic: t = w * inv; u = t + cz (cz = C + zoff, the code's
+// integer lands in the low bits of u); r = u - cz = rint(t); e = t - r
+// (exact); f = e^2 - thr2.  Returns the bits of u and of f for both weights.
+__device__ __forceinline__ void quant_pair(uint32_t h2, uint64_t inv2, uint64_t cz2,
+                                           uint64_t nthr2, uint32_t& u0, uint32_t& u1,
+                                           uint32_t& f0, uint32_t& f1) {
+  asm("{\n\t"
+      ".reg .b16 a, b;\n\t"
+      ".reg .f32 x, y;\n\t"
+      ".reg .b64 w, t, u, r, e, f;\n\t"
+      "mov.b32 {a, b}, %4;\n\t"
+      "cvt.f32.f16 x, a;\n\t"
+      "cvt.f32.f16 y, b;\n\t"
+      "mov.b64 w, {x, y};\n\t"
+      "mul.rn.f32x2 t, w, %5;\n\t"
+      "add.rn.f32x2 u, t, %6;\n\t"
+      "sub.rn.f32x2 r, u, %6;\n\t"
+      "sub.rn.f32x2 e, t, r;\n\t"
+      "fma.rn.f32x2 f, e, e, %7;\n\t"
+      "mov.b64 {%0, %1}, u;\n\t"
+      "mov.b64 {%2, %3}, f;\n\t"
+      "}"
+      : "=r"(u0), "=r"(u1), "=r"(f0), "=r"(f1)
+      : "r"(h2), "l"(inv2), "l"(cz2), "l"(nthr2));
+}
 
-// The exact path of a lane's 32 codes (rint_quotient's tie decision), out of
-// line: it runs only for chunks where some t came within 2^-12 of a
-// half-integer, and keeping it out of the main loop keeps that loop's
-// registers free.
+// The packed word of kPerWord codes at wp with the exact tie rule and both
+// clamps; out of line (it runs only for flagged words), so that the main
+// loop keeps its registers.
 template <int BITS, bool SYM>
-__device__ __noinline__ CodeWords<BITS> exact_codes(uint4 c0, uint4 c1, uint4 c2, uint4 c3,
-                                                    float s, float inv, float z) {
+__device__ __noinline__ uint32_t exact_word(const __half* wp, float s, float inv, float z) {
   constexpr float kQmax = SYM ? float((1 << (BITS - 1)) - 1) : float((1 << BITS) - 1);
   constexpr float kQmin = SYM ? -float(1 << (BITS - 1)) : 0.f;
   constexpr float kOffset = SYM ? float(1 << (BITS - 1)) : 0.f;
   constexpr int kPerWord = 32 / BITS;
-  const uint32_t h[16] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w,
-                          c2.x, c2.y, c2.z, c2.w, c3.x, c3.y, c3.z, c3.w};
-  CodeWords<BITS> out;
+  float q[kPerWord];
 #pragma unroll
-  for (int wi = 0; wi < BITS; ++wi) {
-    float q[kPerWord];
-#pragma unroll
-    for (int e = 0; e < kPerWord; ++e) {
-      const int i = wi * kPerWord + e;
-      const __half2 pair = *reinterpret_cast<const __half2*>(&h[i >> 1]);
-      const float w = (i & 1) ? __high2float(pair) : __low2float(pair);
-      const float r = rint_quotient(w, s, inv);
-      q[e] = SYM ? fminf(fmaxf(r, kQmin), kQmax) + kOffset : fminf(fmaxf(r + z, kQmin), kQmax);
-    }
-    out.w[wi] = pack_codes_f<BITS>(q);
+  for (int e = 0; e < kPerWord; ++e) {
+    const float r = rint_quotient(__half2float(wp[e]), s, inv);
+    q[e] = SYM ? fminf(fmaxf(r, kQmin), kQmax) + kOffset : fminf(fmaxf(r + z, kQmin), kQmax);
   }
-  return out;
+  return pack_codes_f<BITS>(q);
+}
+
+__device__ __forceinline__ uint64_t f32x2_splat(float v) {
+  const uint32_t b = __float_as_uint(v);
+  return (uint64_t(b) << 32) | b;
 }
 
 template <int BITS, bool SYM, int G>
-__global__ void __launch_bounds__(256, 4) quantize2_kernel(const __half* __restrict__ W,
+__global__ void __launch_bounds__(256, 3) quantize2_kernel(const __half* __restrict__ W,
                                                           int64_t total,
                                                           uint8_t* __restrict__ codes,
                                                           __half* __restrict__ scales,
                                                           __half* __restrict__ zeros) {
   static_assert(G % 32 == 0 && G <= 1024, "group must be a multiple of 32");
+  static_assert(BITS == 4 || BITS == 8, "4- or 8-bit codes");
   constexpr int kLanesPerGroup = G / 32;
   constexpr float kQmax = SYM ? float((1 << (BITS - 1)) - 1) : float((1 << BITS) - 1);
+  constexpr float kQmin = SYM ? -float(1 << (BITS - 1)) : 0.f;
   constexpr float kOffset = SYM ? float(1 << (BITS - 1)) : 0.f;
   constexpr int kPerWord = 32 / BITS;  // codes per 32-bit word
   constexpr float kC = 12582912.f;     // 1.5 * 2^23
+  // |t - w/s| <= qmax * 2^-23 < 2^-15; a t farther than 2^-14 from every
+  // half-integer rounds as w/s does, and the clamps cannot bind on it
+  constexpr float kNegThr2 = -0.24993896484375f;  // -(0.5 - 2^-14)^2, rounded
   const int lane = threadIdx.x & 31;
   const int64_t first_warp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t warps = (int64_t(gridDim.x) * blockDim.x) >> 5;
@@ -161,33 +184,51 @@ __global__ void __launch_bounds__(256, 4) quantize2_kernel(const __half* __restr
       if (!SYM) z = fminf(fmaxf(rintf(__fdiv_rn(-lo, s)), 0.f), kQmax);
     }
     const float zoff = SYM ? kOffset : z;  // added to rint(w/s) in the stored code
-    const float cz = kC + zoff;
+    const uint64_t inv2 = f32x2_splat(inv), cz2 = f32x2_splat(kC + zoff);
+    const uint64_t nthr2 = f32x2_splat(kNegThr2);
 
-    // Fast path: codes by the magic-number rounding; the largest distance
-    // of t from its rounded value says whether any tie window was hit.
+    // Fast path: the code is the low byte of u's bits (u - C = rint(t) +
+    // zoff, an integer in [0, 2^b) unless t is near a half-integer); ok
+    // collects, from bit 31 down, whether each weight is clear of the
+    // half-integers (f < 0: sign bit set).
     uint32_t words[BITS];
-    float far = 0.f;
+    uint32_t ok = 0u;
 #pragma unroll
     for (int wi = 0; wi < BITS; ++wi) {
-      float q[kPerWord];
+      uint32_t u[kPerWord];
 #pragma unroll
-      for (int e = 0; e < kPerWord; ++e) {
-        const int i = wi * kPerWord + e;
-        const __half2 pair = *reinterpret_cast<const __half2*>(&h[i >> 1]);
-        const float w = (i & 1) ? __high2float(pair) : __low2float(pair);
-        const float t = w * inv;
-        const float qq = (t + cz) - kC;  // rint(t) + zoff, exact integer
-        far = fmaxf(far, fabsf(t - (qq - zoff)));
-        q[e] = SYM ? qq : fminf(qq, kQmax);
+      for (int pp = 0; pp < kPerWord / 2; ++pp) {
+        uint32_t f0, f1;
+        quant_pair(h[wi * kPerWord / 2 + pp], inv2, cz2, nthr2, u[2 * pp], u[2 * pp + 1], f0, f1);
+        ok = __funnelshift_l(f0, ok, 1);
+        ok = __funnelshift_l(f1, ok, 1);
       }
-      words[wi] = pack_codes_f<BITS>(q);
-    }
-    if (__any_sync(0xffffffffu, far > 0.5f - 0x1p-12f)) {
-      // a t within 2^-12 of a half-integer somewhere in the warp: redo this
-      // lane's codes with the exact tie decision
-      const CodeWords<BITS> ex = exact_codes<BITS, SYM>(cur[0], cur[1], cur[2], cur[3], s, inv, z);
+      if constexpr (BITS == 4) {
+        uint32_t b[4];
 #pragma unroll
-      for (int wi = 0; wi < BITS; ++wi) words[wi] = ex.w[wi];
+        for (int j = 0; j < 4; ++j) b[j] = (u[2 * j + 1] << 4) + u[2 * j];
+        words[wi] = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040),
+                                0x5410);
+      } else {
+        words[wi] = __byte_perm(__byte_perm(u[0], u[1], 0x0040), __byte_perm(u[2], u[3], 0x0040),
+                                0x5410);
+      }
+    }
+    if (__any_sync(0xffffffffu, ok != 0xffffffffu)) {
+      // some t within 2^-14 of a half-integer (in practice w/s exactly on
+      // one): every word holding such a weight is recomputed with the exact
+      // tie decision of quantize.cuh (rint_quotient), from the weights in
+      // global memory
+      constexpr uint32_t kWordBits = ~0u << (32 - kPerWord);
+      uint32_t fl = ~ok;  // bit 31 - i: weight i flagged
+      while (fl != 0u) {
+        const int wi = __clz(fl) / kPerWord;
+        fl &= ~(kWordBits >> (wi * kPerWord));
+        const uint32_t word = exact_word<BITS, SYM>(W + base + wi * kPerWord, s, inv, z);
+#pragma unroll
+        for (int j = 0; j < BITS; ++j)
+          if (j == wi) words[j] = word;
+      }
     }
     if (valid) {
       uint4* dst = reinterpret_cast<uint4*>(codes + base * BITS / 8);

@@ -214,15 +214,19 @@ wq_status wq_matmul(const void* X, int64_t M, const void* codes, const void* sca
     if (!wqh::run_gemm(a, &e)) return WQ_ERR_UNSUPPORTED;
     return from_cuda(e);
   }
-  // Kernel choice (measured on B200, back-to-back launches): the direct-load
-  // kernel wherever it applies (4-bit codes, groups of 128, M <= 4, K a
-  // multiple of 512): faster than both others on every Llama-8B layer shape
-  // at M = 1, 2, 4.  Otherwise: the balanced kernel for 8-bit codes, group
-  // 32, and layers with fewer than three waves of row tiles per SM; the
-  // cluster-split kernel otherwise.  Splitting row tiles across CTAs through
-  // the workspace measured slower than whole tiles on every shape tried (the
-  // end-of-kernel gather costs more than the balance gains), so it is used
-  // only when forced through the tuning hook.
+  // Kernel choice (measured on B200, back-to-back launches from CUDA graphs):
+  // for 4-bit codes in groups of 128 with K = 4096 and M <= 4 the k-sliced
+  // kernel, where the layer has at least one 8-row tile per SM (8.5 us
+  // against 10.2 for the direct-load kernel at N = 14336; slower at N =
+  // 1024); the direct-load kernel wherever it applies (4-bit codes, groups of
+  // 128, M <= 4, K a multiple of 512): faster than both others on every
+  // Llama-8B layer shape at M = 1, 2, 4.  Otherwise: the balanced kernel for
+  // 8-bit codes, group 32, and layers with fewer than three waves of row
+  // tiles per SM; the cluster-split kernel otherwise.  Splitting row tiles
+  // across CTAs through the workspace measured slower than whole tiles on
+  // every shape tried (the end-of-kernel gather costs more than the balance
+  // gains), so it is used only when forced through the tuning hook.
+  if (choice == 0 && N >= 8 * int64_t(a.dev.sms) && wqh::run_ks(a, &e)) return from_cuda(e);
   if (choice == 5) {
     if (wqh::run_tb(a, &e)) return from_cuda(e);
     return WQ_ERR_UNSUPPORTED;
