@@ -140,9 +140,9 @@ size_t wq_matmul_workspace_bytes(void);
  * M > 32 runs the prefill kernel: the exact integers q - z on the tcgen05
  * tensor cores with binary32 accumulators in tensor memory, one per group,
  * scaled by s in binary32 ("量化" (llminference s08) section 实现: large
- * batches are bound by the multiply).  Its scope in this build: group 64 or
- * 128, K a multiple of 64 with K/group a multiple of 8 and at most 256;
- * other formats at M > 32 return WQ_ERR_UNSUPPORTED.
+ * batches are bound by the multiply).  Its scope in this build: groups of
+ * 32, 64 or 128, 4- or 8-bit codes, K a multiple of 128 (a load stage is
+ * 128 k); other shapes at M > 32 return WQ_ERR_UNSUPPORTED.
  *
  * workspace / workspace_bytes: NULL and 0, or a buffer of at least
  * wq_matmul_workspace_bytes() bytes as described there.  With it, every SM

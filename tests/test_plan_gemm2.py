@@ -1,9 +1,10 @@
 """Host-side check of the plan of the prefill kernel that keeps the
 dequantized weights in tensor memory (gemm2.cuh): shared-memory rings in
 bounds and 1024-byte aligned (the 128-byte swizzle of the activation boxes
-and the 32/64-byte swizzle of the code boxes), copy boxes inside the TMA
+and the 64/128-byte swizzle of the code boxes), copy boxes inside the TMA
 limits with 16-byte aligned inner extents, the tile count and persistent
-grid, and the kernel's scope (groups 32/64/128, K a multiple of 64)."""
+grid, and the kernel's scope (groups 32/64/128, K a multiple of 128: a load
+stage is 128 k, eight MMAs of K = 16)."""
 import ctypes
 import os
 
@@ -15,7 +16,7 @@ FIELDS = ["M", "N", "K", "ngroups", "tiles_t", "tiles_w", "num_tiles", "codes_st
           "smem", "grid"]
 SMEM_OPTIN, SMS = 232448, 148
 BW = 128
-BK, HEAD = 64, 1024
+BK, HEAD = 128, 1024
 
 
 @pytest.fixture(scope="module")
@@ -50,14 +51,17 @@ def test_plan_gemm2(lib, M, N, K, bits, group):
     assert p["tiles_t"] == -(-M // BT) and p["tiles_w"] == -(-N // BW)
     assert p["num_tiles"] == p["tiles_t"] * p["tiles_w"]
     assert p["grid"] == min(p["num_tiles"], SMS)
-    # code boxes: 128 rows x (64 k of codes) = 32 or 64 bytes per row, a
-    # multiple of 16 bytes, swizzled 32B / 64B; stage size a multiple of 1 KB
+    # code boxes: 128 rows x (128 k of codes) = 64 or 128 bytes per row, a
+    # multiple of 16 bytes, swizzled 64B / 128B (the swizzle span covers the
+    # row); stage size a multiple of 1 KB
     row = BK * bits // 8
-    assert row % 16 == 0 and row in (32, 64)
+    assert row % 16 == 0 and row in (64, 128)
     assert p["codes_stage_bytes"] == BW * row and p["codes_stage_bytes"] % 1024 == 0
-    # activation boxes: 64 k x BT tokens of bfloat16, 128-byte rows
-    x_stage = BT * BK * 2
-    assert x_stage % 1024 == 0
+    # activation stage: two boxes of 64 k x BT tokens of bfloat16 (128-byte
+    # rows, the 128-byte swizzle's span), each 1024-byte aligned
+    x_box = BT * 64 * 2
+    x_stage = 2 * x_box
+    assert x_box % 1024 == 0 and x_stage == BT * BK * 2
     off_codes = HEAD + STAGES * x_stage
     assert off_codes % 1024 == 0
     # the ring of scale / zero blocks (8 slots of 128 rows x 8 groups x 2
@@ -65,15 +69,16 @@ def test_plan_gemm2(lib, M, N, K, bits, group):
     meta = 8 * 2 * 128 * 8 * 2 if (K // group) % 8 == 0 else 0
     assert (off_codes + STAGES * p["codes_stage_bytes"]) % 128 == 0
     assert p["smem"] == off_codes + STAGES * p["codes_stage_bytes"] + meta <= SMEM_OPTIN
-    # every TMA x coordinate (k * 2 bytes for X, bytes for the codes) stays a
-    # multiple of 16 bytes
-    assert (BK * 2) % 16 == 0 and row % 16 == 0
+    # every TMA x coordinate (k * 2 bytes for X: stage start and start + 64;
+    # bytes for the codes) stays a multiple of 16 bytes
+    assert (BK * 2) % 16 == 0 and (64 * 2) % 16 == 0 and row % 16 == 0
     # the code tensor's row pitch is a multiple of 16 bytes (TMA stride rule)
     assert (K * bits // 8) % 16 == 0
 
 
 @pytest.mark.parametrize("M,N,K,bits,group", [(64, 256, 4128, 4, 32), (64, 256, 96, 4, 32),
+                                              (64, 256, 4160, 4, 32), (129, 256, 192, 8, 64),
                                               (64, 256, 4096, 2, 128)])
 def test_out_of_scope(lib, M, N, K, bits, group):
-    # K not a multiple of 64; unsupported code width
+    # K not a multiple of 128; unsupported code width
     assert plan(lib, M, N, K, bits, group) is None

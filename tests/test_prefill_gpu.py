@@ -8,7 +8,7 @@ one-hot activations bit-exact (each output is one exact product s (q - z)).
 Every test runs on both prefill kernels: the one with both operands in
 shared memory ("shared", groups of 64 or 128 with a multiple of 8 groups per
 row) and the one with the dequantized weights in tensor memory ("tmem",
-every group size, K a multiple of 64)."""
+every group size, K a multiple of 128)."""
 import ctypes
 
 import numpy as np
@@ -36,7 +36,7 @@ def kernel(request):
 def in_scope(kernel, K, group):
     if kernel == "shared":
         return group in (64, 128) and (K // group) % 8 == 0 and K // group <= 256
-    return K % 64 == 0
+    return K % 128 == 0
 
 
 def quantize_both(W, bits, group, sym, key=None):

@@ -248,6 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   auto wait = [&](int bar, uint32_t parity) {
+    if (mbar_test_wait(&bars[bar], parity)) return true;  // completed: no flag read
     if (*abort_flag) return false;
     if (!mbar_wait(&bars[bar], parity)) {
       *abort_flag = 1;

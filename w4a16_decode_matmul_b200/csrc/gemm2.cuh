@@ -57,16 +57,17 @@ using gemm::tmem_wait_ld;
 using gemm::umma_desc_sw128;
 
 constexpr int kBW = 128;     // rows of W per tile (MMA M)
-constexpr int kBK = 64;      // k per load stage
+constexpr int kBK = 128;     // k per load stage (8 MMAs of K = 16)
 constexpr int kMaxLoadStages = 8;
-constexpr int kAStages = 8;  // 32-column A stages in tensor memory
+constexpr int kMaxAStages = 8;  // barrier slots for A stages in tensor memory
 constexpr int kDequantWarp0 = 2;
 // threads of a CTA with DW dequantize and EW epilogue warps (and the
 // producer and MMA warps)
 __host__ __device__ constexpr int threads_for(int dw, int ew) { return (2 + dw + ew) * 32; }
 constexpr int kTmemCols = 512;
-constexpr int kAStageCols = kBK / 2;              // 64 k of bfloat16 pairs
-// Bytes of one activation stage (BT tokens x 64 k of bfloat16).
+constexpr int kAStageCols = kBK / 2;              // 128 k of bfloat16 pairs
+// Bytes of one activation stage (BT tokens x 128 k of bfloat16: two boxes
+// of 64 k, as the 128-byte swizzle spans 64 bfloat16).
 __host__ __device__ constexpr int x_stage_bytes(int bt) { return bt * kBK * 2; }
 // Instruction descriptor: binary32 accumulator, bfloat16 A and B, both
 // K-major, N = BT tokens, M = 128 rows of W.
@@ -78,8 +79,8 @@ __host__ __device__ constexpr uint32_t instr_desc(int bt) {
 // mbarrier slots (8 bytes each) in the first KB of shared memory
 constexpr int kBarFull = 0;                    // [kMaxLoadStages] X + codes landed (tx)
 constexpr int kBarEmpty = 8;                   // [kMaxLoadStages] MMAs + dequantize done
-constexpr int kBarAFull = 16;                  // [kAStages] A stage written
-constexpr int kBarAEmpty = 24;                 // [kAStages] A stage read by the MMAs
+constexpr int kBarAFull = 16;                  // [kMaxAStages] A stage written
+constexpr int kBarAEmpty = 24;                 // [kMaxAStages] A stage read by the MMAs
 constexpr int kBarDFull = 32;                  // [2] group accumulator ready
 constexpr int kBarDEmpty = 34;                 // [2] group accumulator read
 constexpr int kBarMmaDone = 36;                // every MMA of the CTA finished
@@ -228,12 +229,16 @@ __global__ void __launch_bounds__(threads_for(DW, EW), 1)
   constexpr int kXStageBytes = x_stage_bytes(BT);
   constexpr int kDCols = BT;                       // one group accumulator
   constexpr int kACol0 = 2 * kDCols;               // A stages after the two accumulators
+  // A stages of 64 columns in the rest of tensor memory: 4 (BT = 128), 6 (BT = 64)
+  constexpr int kAStages = (kTmemCols - kACol0) / kAStageCols;
+  static_assert(kAStages >= 2 && kAStages <= kMaxAStages, "A stages");
+  constexpr int kXBoxBytes = BT * 64 * 2;          // one 64-k activation box
   constexpr uint32_t kIdesc = instr_desc(BT);
   constexpr int kEpiCols = kBT / (EW / 4);         // tokens per epilogue thread
   constexpr int kStagesPerBlock = kMetaGroups * G / kBK;  // load stages per metadata block
   constexpr int kStepsPerGroup = G / 16;        // 16-k MMA steps per group
-  constexpr int kCodesRowBytes = kBK * BITS / 8;  // 32 | 64 bytes of a row per stage
-  constexpr int kChunks = kCodesRowBytes / 16;     // 2 | 4 chunks of 16 bytes
+  constexpr int kCodesRowBytes = kBK * BITS / 8;  // 64 | 128 bytes of a row per stage
+  constexpr int kChunks = kCodesRowBytes / 16;     // 4 | 8 chunks of 16 bytes
   constexpr int kMyChunks = kChunks * 4 / DW;      // chunks of a row per dequantize thread
   constexpr int kMyCols = kAStageCols * 4 / DW;    // A columns per dequantize thread
 
@@ -280,6 +285,7 @@ __global__ void __launch_bounds__(threads_for(DW, EW), 1)
   const uint32_t tmem_base = *tmem_slot;
 
   auto wait = [&](int bar, uint32_t parity) {
+    if (mbar_test_wait(&bars[bar], parity)) return true;  // completed: no flag read
     if (*abort_flag) return false;
     if (!mbar_wait(&bars[bar], parity)) {
       *abort_flag = 1;
@@ -329,6 +335,8 @@ __global__ void __launch_bounds__(threads_for(DW, EW), 1)
           mbar_arrive_expect_tx(&bars[kBarFull + s], uint32_t(kXStageBytes) + p.codes_stage_bytes);
           tma_load_2d(smem + p.off_x + s * kXStageBytes, &tm_x, &bars[kBarFull + s], kb * kBK,
                       t0, keep);
+          tma_load_2d(smem + p.off_x + s * kXStageBytes + kXBoxBytes, &tm_x, &bars[kBarFull + s],
+                      kb * kBK + 64, t0, keep);
           tma_load_2d(smem + p.off_codes + s * p.codes_stage_bytes, &tm_codes,
                       &bars[kBarFull + s], kb * kCodesRowBytes, w0, keep);
         }
@@ -371,7 +379,9 @@ __global__ void __launch_bounds__(threads_for(DW, EW), 1)
               tc_fence_after();
               d = tmem_base + uint32_t(db * kDCols);
             }
-            tc_mma_ts(d, a_addr + uint32_t(8 * k), xdesc + uint64_t(2 * k), kIdesc,
+            // k step k: box k / 4 of the stage, 32 bytes further per step in it
+            tc_mma_ts(d, a_addr + uint32_t(8 * k),
+                      xdesc + uint64_t((k / 4) * (kXBoxBytes >> 4) + 2 * (k % 4)), kIdesc,
                       step_in_group > 0 ? 1u : 0u);
             if (++step_in_group == kStepsPerGroup) {
               tc_commit(&bars[kBarDFull + (gcount & 1)]);
@@ -427,10 +437,10 @@ __global__ void __launch_bounds__(threads_for(DW, EW), 1)
                 r * kMetaGroups;
         }
         // the stage's codes of row r, unswizzled: chunk c sits at chunk
-        // c ^ key (32-byte swizzle: bit 4 of the address XOR bit 7; 64-byte
-        // swizzle: bits 4-5 XOR bits 7-8)
+        // c ^ key (64-byte swizzle: bits 4-5 of the address XOR bits 7-8;
+        // 128-byte swizzle: bits 4-6 XOR bits 7-9)
         const uint8_t* crow = smem + p.off_codes + s * p.codes_stage_bytes + r * kCodesRowBytes;
-        const int key = kChunks == 2 ? ((r >> 2) & 1) : ((r >> 1) & 3);
+        const int key = kChunks == 4 ? ((r >> 1) & 3) : (r & 7);
         uint32_t o[kMyCols];
         if constexpr (BITS == 4) {
 #pragma unroll
@@ -482,7 +492,16 @@ __global__ void __launch_bounds__(threads_for(DW, EW), 1)
           ++mb;
         }
         const uint32_t col = uint32_t(kACol0 + as * kAStageCols + part * kMyCols);
-        if constexpr (kMyCols == 32) {
+        if constexpr (kMyCols == 64) {
+          uint32_t lo[32], hi[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            lo[i] = o[i];
+            hi[i] = o[32 + i];
+          }
+          tmem_st32(tmem_base + lanes + col, lo);
+          tmem_st32(tmem_base + lanes + col + 32, hi);
+        } else if constexpr (kMyCols == 32) {
           tmem_st32(tmem_base + lanes + col, o);
         } else {
           tmem_st16(tmem_base + lanes + col, o);

@@ -22,11 +22,11 @@ struct Gemm2Plan {
 struct Gemm2Variant {
   int load_stages, dequant_warps, epilogue_warps;
 };
-constexpr Gemm2Variant kGemm2Variants[] = {{4, 4, 8}, {8, 4, 8}, {6, 4, 16}};
+constexpr Gemm2Variant kGemm2Variants[] = {{4, 4, 8}, {3, 4, 8}, {4, 8, 8}};
 constexpr int kNumGemm2Variants = int(sizeof(kGemm2Variants) / sizeof(kGemm2Variants[0]));
 int g_gemm2_variant = 0;
 
-// Scope: groups of 32, 64 or 128, K a multiple of 64; any M and N.
+// Scope: groups of 32, 64 or 128, K a multiple of 128; any M and N.
 bool plan_gemm2(int M, int N, int K, int bits, int group, const DeviceInfo& dev,
                 Gemm2Plan* plan, int variant) {
   using namespace wq::gemm2;
@@ -74,18 +74,18 @@ cudaError_t launch_gemm2(Gemm2Plan* plan, const DeviceInfo* dev, const void* X, 
   }
   const wq::gemm2::Params& p = plan->p;
   CUtensorMap tx, tc;
-  // X [M][K] bfloat16, boxes of 64 k x BT tokens, 128-byte swizzle (the
+  // X [M][K] bfloat16, boxes of 64 k x BT tokens (two per 128-k stage), 128-byte swizzle (the
   // K-major canonical layout of the MMA's B operand)
   if (!encode_2d_ex(&tx, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, uint64_t(p.K), uint64_t(p.M),
-                    uint32_t(kBK), uint32_t(BT), CU_TENSOR_MAP_SWIZZLE_128B,
+                    64u, uint32_t(BT), CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
     return cudaErrorInvalidValue;
-  // codes [N][K*bits/8] bytes, boxes of 64 k x 128 rows, swizzled so that
+  // codes [N][K*bits/8] bytes, boxes of 128 k x 128 rows, swizzled so that
   // the dequantize threads (one row each) read without bank conflicts
   const uint32_t row_box = uint32_t(kBK * BITS / 8);
   if (!encode_2d_ex(&tc, c, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(p.K) * BITS / 8,
                     uint64_t(p.N), row_box, uint32_t(kBW),
-                    BITS == 4 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B,
+                    BITS == 4 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
     return cudaErrorInvalidValue;
   // scales / zeros [N][ngroups] binary16, boxes of 8 groups x 128 rows
@@ -109,8 +109,8 @@ cudaError_t launch_gemm2_v(Gemm2Plan* plan, const DeviceInfo* dev, const void* X
                            const void* sc, const void* z, cudaStream_t s) {
   if (plan->bt == 64) return launch_gemm2<BITS, SYM, G, 6, 4, 8, 64, MT>(plan, dev, X, c, sc, z, s);
   switch (plan->variant) {
-    case 1: return launch_gemm2<BITS, SYM, G, 8, 4, 8, 128, MT>(plan, dev, X, c, sc, z, s);
-    case 2: return launch_gemm2<BITS, SYM, G, 6, 4, 16, 128, MT>(plan, dev, X, c, sc, z, s);
+    case 1: return launch_gemm2<BITS, SYM, G, 3, 4, 8, 128, MT>(plan, dev, X, c, sc, z, s);
+    case 2: return launch_gemm2<BITS, SYM, G, 4, 8, 8, 128, MT>(plan, dev, X, c, sc, z, s);
     default: return launch_gemm2<BITS, SYM, G, 4, 4, 8, 128, MT>(plan, dev, X, c, sc, z, s);
   }
 }

@@ -40,7 +40,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }  // namespace
 
 int g_kernel_choice = 0;
-int g_prefill_choice = 1;
+int g_prefill_choice = 0;  // 0: tensor-memory kernel first (measured faster at every M), then shared
 
 bool device_info(DeviceInfo* out) {
   int dev = 0;
