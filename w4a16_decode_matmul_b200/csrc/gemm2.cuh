@@ -23,8 +23,12 @@
 //
 // Persistent CTAs walk 128 x 128 tiles (token tile major, so that the CTAs of
 // a wave share one activation tile and the whole weight matrix stays in L2).
-// A load stage is 64 k: the activation box (128 tokens x 64 k, 128-byte
-// swizzle, K-major) and the codes box (128 rows x 64 k of codes, swizzled).
+// A load stage is 128 k: two activation boxes (128 tokens x 64 k, 128-byte
+// swizzle, K-major) and the codes box (128 rows x 128 k of codes, 64- or
+// 128-byte swizzle).  128 k is eight MMAs per barrier hand-off: with four
+// (64 k) the issuing thread's per-stage wait and commit left the tensor pipe
+// idle most of the time (measured on B200: ~240 cycles per 64-cycle MMA
+// against ~90 with eight per stage).
 // Warp roles:
 //   warp 0      TMA producer (one thread);
 //   warp 1      tensor-memory allocation; one thread issues tcgen05.mma
@@ -32,8 +36,9 @@
 //               in shared memory, into one of two 128-column group
 //               accumulators, and commits it to the epilogue after a group;
 //   warps 2-5   dequantize: one row of W per thread; a stage's codes ->
-//               32 columns of bfloat16 pairs (q - z) -> tensor memory
-//               (one of eight 32-column A stages);
+//               64 columns of bfloat16 pairs (q - z) -> tensor memory
+//               (A stage s sits beside load stage s: both are freed by the
+//               one commit of the stage's MMAs);
 //   warps 6-13  epilogue: one row of W and 64 tokens per thread; per group
 //               S += s_g D_g in registers; S is written to Y at the end of
 //               the tile.
@@ -80,7 +85,6 @@ __host__ __device__ constexpr uint32_t instr_desc(int bt) {
 constexpr int kBarFull = 0;                    // [kMaxLoadStages] X + codes landed (tx)
 constexpr int kBarEmpty = 8;                   // [kMaxLoadStages] MMAs + dequantize done
 constexpr int kBarAFull = 16;                  // [kMaxAStages] A stage written
-constexpr int kBarAEmpty = 24;                 // [kMaxAStages] A stage read by the MMAs
 constexpr int kBarDFull = 32;                  // [2] group accumulator ready
 constexpr int kBarDEmpty = 34;                 // [2] group accumulator read
 constexpr int kBarMmaDone = 36;                // every MMA of the CTA finished
@@ -232,6 +236,7 @@ __global__ void __launch_bounds__(threads_for(DW, EW), 1)
   // A stages of 64 columns in the rest of tensor memory: 4 (BT = 128), 6 (BT = 64)
   constexpr int kAStages = (kTmemCols - kACol0) / kAStageCols;
   static_assert(kAStages >= 2 && kAStages <= kMaxAStages, "A stages");
+  static_assert(LS == kAStages, "one ring: load stage s and A stage s are freed together");
   constexpr int kXBoxBytes = BT * 64 * 2;          // one 64-k activation box
   constexpr uint32_t kIdesc = instr_desc(BT);
   constexpr int kEpiCols = kBT / (EW / 4);         // tokens per epilogue thread
@@ -258,7 +263,6 @@ __global__ void __launch_bounds__(threads_for(DW, EW), 1)
     }
     for (int s = 0; s < kAStages; ++s) {
       mbar_init(&bars[kBarAFull + s], kNumDequantWarps);
-      mbar_init(&bars[kBarAEmpty + s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars[kBarDFull + b], 1);
@@ -359,9 +363,10 @@ __global__ void __launch_bounds__(threads_for(DW, EW), 1)
         uint32_t d = 0;
         for (int kb = 0; kb < nkb && !stop; ++kb, ++ld) {
           const int s = ld % kLoadStages;
-          const int as = ld % kAStages;
-          if (!wait(kBarFull + s, uint32_t(ld / kLoadStages) & 1u) ||
-              !wait(kBarAFull + as, uint32_t(ld / kAStages) & 1u)) {
+          const int as = s;  // the A stages are the load stages' slots
+          // A written implies the stage's activations landed: the dequantize
+          // warps wait for the stage's copies before they arrive here
+          if (!wait(kBarAFull + as, uint32_t(ld / kAStages) & 1u)) {
             stop = true;
             break;
           }
@@ -390,9 +395,9 @@ __global__ void __launch_bounds__(threads_for(DW, EW), 1)
             }
           }
           if (stop) break;
-          // the stage's activations and A columns are free once these MMAs finish
+          // the stage's activations, codes and A columns are free once these
+          // MMAs finish (one commit: the A stages are the load stages' slots)
           tc_commit(&bars[kBarEmpty + s]);
-          tc_commit(&bars[kBarAEmpty + as]);
         }
       }
       // all MMAs of this CTA complete before tensor memory is freed
@@ -417,8 +422,9 @@ __global__ void __launch_bounds__(threads_for(DW, EW), 1)
       for (int kb = 0; kb < nkb; ++kb, ++ld) {
         const int s = ld % kLoadStages;
         const int as = ld % kAStages;
-        if (!wait(kBarFull + s, uint32_t(ld / kLoadStages) & 1u) ||
-            !wait(kBarAEmpty + as, (uint32_t(ld / kAStages) & 1u) ^ 1u)) {
+        // the stage's copies landed; then A stage `as` is free as well: the
+        // copies were issued after the MMAs of its previous use committed
+        if (!wait(kBarFull + s, uint32_t(ld / kLoadStages) & 1u)) {
           stop = true;
           break;
         }

@@ -166,9 +166,14 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_ks_kernel(const Params p) {
   const int gi = 2 * pair + hh;
   // this lane's two table entries for the first tile; successive tiles are
   // 8 rows further
-  const float2* szp = sz + rr0 * kSzStride + gi;
-  float* dst = part + size_t(warp) * per_tile;
-  const size_t part_tile_stride = size_t(kWarps) * per_tile;
+  // 32-bit shared addresses: this lane's two table entries for the first
+  // tile (successive tiles are 8 rows further) and its partial-sum slots
+  const int mrow = MT == 1 ? 1 : p.M;
+  uint32_t sz_a = smem_addr(sz + rr0 * kSzStride + gi);
+  uint32_t dst0 = smem_addr(part + warp * per_tile + rr0 * mrow + m0);
+  uint32_t dst1 = smem_addr(part + warp * per_tile + rr0 * mrow + (m1 & 3));
+  const uint32_t part_tile_bytes = uint32_t(kWarps * per_tile) * 4u;
+  const uint32_t row4_bytes = uint32_t(4 * mrow) * 4u;
   // the partial sums of this warp's slots: every slot of every tile is
   // written below (rows past N included), so no clearing is needed; the
   // {s, 128 + z} table was written by all threads
@@ -177,7 +182,6 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_ks_kernel(const Params p) {
   // Every lane computes its epilogue values (a lane and its partner L ^ 6
   // are both owners or both not; only owners' sums are stored), so the loop
   // has no branch but its end; slots are compile-time constants.
-  const int mrow = MT == 1 ? 1 : p.M;
   const bool st0 = hh == 0 && use0, st1 = hh == 0 && use1;
   for (int it0 = 0; it0 < ntiles; it0 += DEPTH) {
 #pragma unroll
@@ -207,16 +211,18 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_ks_kernel(const Params p) {
       // y = s (C - (128 + z) Sx) for tile rows rr0 and rr0 + 4, in binary32;
       // the row's two groups are then added (lanes L and L ^ 6; binary32
       // addition commutes, so both lanes hold the same sum)
-      const float2 e0 = szp[0];
-      const float2 e1 = szp[4 * kSzStride];
-      szp += kTileRows * kSzStride;
+      const uint2 e0b = lds64(sz_a);
+      const uint2 e1b = lds64(sz_a + 4 * kSzStride * 8);
+      sz_a += kTileRows * kSzStride * 8;
+      const float2 e0 = make_float2(__uint_as_float(e0b.x), __uint_as_float(e0b.y));
+      const float2 e1 = make_float2(__uint_as_float(e1b.x), __uint_as_float(e1b.y));
       float y0 = e0.x * fmaf(-e0.y, sx0, d[0]);
       float y2 = e1.x * fmaf(-e1.y, sx0, d[2]);
       y0 += __shfl_xor_sync(0xffffffffu, y0, 6);
       y2 += __shfl_xor_sync(0xffffffffu, y2, 6);
       if (st0) {
-        dst[rr0 * mrow + m0] = y0;
-        dst[(rr0 + 4) * mrow + m0] = y2;
+        sts32(dst0, y0);
+        sts32(dst0 + row4_bytes, y2);
       }
       if constexpr (MT > 1) {
         float y1 = e0.x * fmaf(-e0.y, sx1, d[1]);
@@ -224,11 +230,12 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_ks_kernel(const Params p) {
         y1 += __shfl_xor_sync(0xffffffffu, y1, 6);
         y3 += __shfl_xor_sync(0xffffffffu, y3, 6);
         if (st1) {
-          dst[rr0 * mrow + m1] = y1;
-          dst[(rr0 + 4) * mrow + m1] = y3;
+          sts32(dst1, y1);
+          sts32(dst1 + row4_bytes, y3);
         }
       }
-      dst += part_tile_stride;
+      dst0 += part_tile_bytes;
+      dst1 += part_tile_bytes;
     }
   }
   ld::cp_async_wait<0>();

@@ -22,7 +22,7 @@ struct Gemm2Plan {
 struct Gemm2Variant {
   int load_stages, dequant_warps, epilogue_warps;
 };
-constexpr Gemm2Variant kGemm2Variants[] = {{4, 4, 8}, {3, 4, 8}, {4, 8, 8}};
+constexpr Gemm2Variant kGemm2Variants[] = {{4, 4, 8}, {4, 4, 16}, {4, 8, 8}};
 constexpr int kNumGemm2Variants = int(sizeof(kGemm2Variants) / sizeof(kGemm2Variants[0]));
 int g_gemm2_variant = 0;
 
@@ -109,7 +109,7 @@ cudaError_t launch_gemm2_v(Gemm2Plan* plan, const DeviceInfo* dev, const void* X
                            const void* sc, const void* z, cudaStream_t s) {
   if (plan->bt == 64) return launch_gemm2<BITS, SYM, G, 6, 4, 8, 64, MT>(plan, dev, X, c, sc, z, s);
   switch (plan->variant) {
-    case 1: return launch_gemm2<BITS, SYM, G, 3, 4, 8, 128, MT>(plan, dev, X, c, sc, z, s);
+    case 1: return launch_gemm2<BITS, SYM, G, 4, 4, 16, 128, MT>(plan, dev, X, c, sc, z, s);
     case 2: return launch_gemm2<BITS, SYM, G, 4, 8, 8, 128, MT>(plan, dev, X, c, sc, z, s);
     default: return launch_gemm2<BITS, SYM, G, 4, 4, 8, 128, MT>(plan, dev, X, c, sc, z, s);
   }
