@@ -615,11 +615,11 @@ def q4k_point(wq, torch, dev, stream, reps: int = 10):
     Y = torch.empty(M, N, dtype=torch.float32, device=dev)
     g = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
-        wq.q4k_matmul(X, pool[0], N, K, out=Y)
+        wq.q4k_matmul(X, pool[0], N, K, out=Y, static_weights=True)
         stream.synchronize()
         with torch.cuda.graph(g, stream=stream):
             for b in pool:
-                wq.q4k_matmul(X, b, N, K, out=Y)
+                wq.q4k_matmul(X, b, N, K, out=Y, static_weights=True)
         g.replay()
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s.record(stream)
@@ -633,7 +633,8 @@ def q4k_point(wq, torch, dev, stream, reps: int = 10):
     return {"us_per_layer": round(us, 3), "gbs": round(moved / us / 1e3, 1),
             "bytes_per_layer": moved, "frac": round(moved / us / 1e3 / peak, 4),
             "peak_kind": f"{kind} HBM copy",
-            "how": f"M=1, K={K}, N={N}, 144-byte superblocks (4.5 bits per weight), CUDA "
+            "how": f"M=1, K={K}, N={N}, 144-byte superblocks (4.5 bits per weight), static "
+                   f"weights (programmatic dependent launch), CUDA "
                    f"graph of {pool_n} launches over rotating copies"}
 
 

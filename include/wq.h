@@ -226,6 +226,16 @@ wq_status wq_q4k_quantize(const void *W, int64_t N, int64_t K, void *blocks,
 wq_status wq_q4k_matmul(const void *X, int64_t M, const void *blocks, int64_t N, int64_t K,
                         void *Y, int out_dtype, wq_stream_t stream);
 
+/* As wq_q4k_matmul, with flags: 0 or WQ_MATMUL_STATIC_WEIGHTS, which means
+ * as for wq_matmul that nothing enqueued before the call on `stream` writes
+ * the blocks: the kernel is launched as a programmatic dependent of the
+ * previous work and may read the blocks before that work has finished (X and
+ * Y only after).  Errors as wq_q4k_matmul, and WQ_ERR_INVALID_ARG for an
+ * unknown flag. */
+wq_status wq_q4k_matmul_ex(const void *X, int64_t M, const void *blocks, int64_t N,
+                           int64_t K, void *Y, int out_dtype, unsigned int flags,
+                           wq_stream_t stream);
+
 /* Read and clear the device status word (WQ_OK if no kernel recorded an
  * error).  Synchronizes `stream` first. */
 wq_status wq_get_device_error(wq_stream_t stream);

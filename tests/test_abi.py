@@ -83,6 +83,11 @@ def test_superblock_rejections_without_gpu(lib):
     assert lib.wq_q4k_matmul(base, 9, base, 4, 256, base, 0, None) == 1   # M > 8
     assert lib.wq_q4k_matmul(base, 1, base, 4, 256, base, 7, None) == 1   # out dtype
     assert lib.wq_q4k_matmul(base, 1, base + 8, 4, 256, base, 0, None) == 3
+    lib.wq_q4k_matmul_ex.argtypes = [vp, i64, vp, i64, i64, vp, ctypes.c_int, ctypes.c_uint, vp]
+    lib.wq_q4k_matmul_ex.restype = ctypes.c_int
+    assert lib.wq_q4k_matmul_ex(base, 1, base, 4, 256, base, 0, 2, None) == 1   # unknown flag
+    assert lib.wq_q4k_matmul_ex(base, 9, base, 4, 256, base, 0, 1, None) == 1   # M > 8
+    assert lib.wq_q4k_matmul_ex(base, 1, base + 8, 4, 256, base, 0, 1, None) == 3
 
 
 def test_status_strings(lib):

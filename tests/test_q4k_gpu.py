@@ -3,6 +3,8 @@ the quantizer's blocks bit-exact (tiny, ragged-row, edge-value and full
 Llama-8B layer shapes), and the fused small-batch matmul within
 |y - y_ref| <= 1e-4 sum|x w| (+ one bfloat16 ulp for bfloat16 out), with
 y_ref the binary64 product of X and the oracle's reconstruction."""
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -70,6 +72,37 @@ def test_matmul_tolerance(M, N, K):
     torch.cuda.synchronize()
     check_tolerance(Y.cpu().numpy()[:, rows], y_ref, y_abs, False)
     check_tolerance(Yb.float().cpu().numpy()[:, rows], y_ref, y_abs, True)
+
+
+@pytest.mark.parametrize("N", [1, 15, 16, 17, 1000, 2323, 14336])
+@pytest.mark.parametrize("kernel", [0, 1])
+def test_kernels_at_k4096(N, kernel):
+    """M = 1, K = 4096 runs the tensor-core kernel (16-row tiles, one warp per
+    superblock; ragged N exercises the zero-filled rows of the last tile);
+    the tuning hook forces the scalar kernel.  Both against the oracle, and
+    bit-identical between a plain call and one with static weights
+    (programmatic dependent launch)."""
+    K = 4096
+    lib = wq().lib
+    lib.wq_internal_set_q4k_kernel.argtypes = [ctypes.c_int]
+    lib.wq_internal_set_q4k_kernel(kernel)
+    try:
+        W = synth.weight(N, K, seed=3 * N + 7)
+        X = synth.activation(1, K, seed=N + 11)
+        blocks, ref = quantize_both(W)
+        rng = np.random.default_rng(N)
+        rows = np.unique(np.r_[np.arange(min(N, 40)), np.arange(max(0, N - 40), N),
+                               rng.integers(0, N, 200)])
+        y_ref, y_abs = sampled_reference(X, ref, N, K, rows)
+        Y = wq().q4k_matmul(X.cuda(), blocks, N, K)
+        Y2 = wq().q4k_matmul(X.cuda(), blocks, N, K, static_weights=True)
+        Yb = wq().q4k_matmul(X.cuda(), blocks, N, K, out_dtype=torch.bfloat16)
+        torch.cuda.synchronize()
+        assert torch.equal(Y, Y2)
+        check_tolerance(Y.cpu().numpy()[:, rows], y_ref, y_abs, False)
+        check_tolerance(Yb.float().cpu().numpy()[:, rows], y_ref, y_abs, True)
+    finally:
+        lib.wq_internal_set_q4k_kernel(0)
 
 
 def test_matmul_deterministic_and_one_hot():

@@ -72,6 +72,8 @@ def _load() -> ctypes.CDLL:
     lib.wq_q4k_quantize.restype = i32
     lib.wq_q4k_matmul.argtypes = [vp, i64, vp, i64, i64, vp, i32, vp]
     lib.wq_q4k_matmul.restype = i32
+    lib.wq_q4k_matmul_ex.argtypes = [vp, i64, vp, i64, i64, vp, i32, ctypes.c_uint, vp]
+    lib.wq_q4k_matmul_ex.restype = i32
     lib.wq_get_device_error.argtypes = [vp]
     lib.wq_get_device_error.restype = i32
     lib.wq_status_string.argtypes = [i32]
@@ -270,9 +272,11 @@ def q4k_quantize(W: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tens
 
 def q4k_matmul(X: torch.Tensor, blocks: torch.Tensor, N: int, K: int,
                out_dtype: torch.dtype = torch.float32,
-               out: torch.Tensor | None = None) -> torch.Tensor:
-    """``wq_q4k_matmul``: Y [M, N] = X [M, K] (bfloat16, M <= 8) times What^T
-    for superblock weights; X, blocks and Y on the GPU."""
+               out: torch.Tensor | None = None, static_weights: bool = False) -> torch.Tensor:
+    """``wq_q4k_matmul_ex``: Y [M, N] = X [M, K] (bfloat16, M <= 8) times What^T
+    for superblock weights; X, blocks and Y on the GPU.  ``static_weights``
+    passes WQ_MATMUL_STATIC_WEIGHTS (nothing enqueued before writes the
+    blocks)."""
     if X.dtype != torch.bfloat16 or X.dim() != 2 or X.shape[1] != K:
         raise ValueError("X must be a 2-D bfloat16 tensor [M, K]")
     if out_dtype not in (torch.float32, torch.bfloat16):
@@ -281,9 +285,10 @@ def q4k_matmul(X: torch.Tensor, blocks: torch.Tensor, N: int, K: int,
     Y = out if out is not None else torch.empty((M, N), dtype=out_dtype, device=X.device)
     dev = _require_cuda(X, blocks, Y)
     with torch.cuda.device(dev):
-        _check(lib.wq_q4k_matmul(_ptr(X), M, _ptr(blocks), N, K, _ptr(Y),
-                                 WQ_OUT_BF16 if Y.dtype == torch.bfloat16 else WQ_OUT_F32,
-                                 _stream(dev)), "wq_q4k_matmul")
+        _check(lib.wq_q4k_matmul_ex(_ptr(X), M, _ptr(blocks), N, K, _ptr(Y),
+                                    WQ_OUT_BF16 if Y.dtype == torch.bfloat16 else WQ_OUT_F32,
+                                    WQ_MATMUL_STATIC_WEIGHTS if static_weights else 0,
+                                    _stream(dev)), "wq_q4k_matmul_ex")
     return Y
 
 

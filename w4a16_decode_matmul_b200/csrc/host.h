@@ -90,7 +90,7 @@ cudaError_t run_dequantize(int bits, bool sym, int group, const void* codes, con
 cudaError_t run_q4k_quantize(const void* W, int64_t nblocks, void* blocks, cudaStream_t s,
                              int sms);
 cudaError_t run_q4k_matmul(const void* X, int M, const void* blocks, int N, int K, void* Y,
-                           bool y_bf16, cudaStream_t s, int sms);
+                           bool y_bf16, bool pdl, cudaStream_t s, int sms);
 
 // Balanced-kernel workspace geometry (flags, then partial sums).
 size_t sk_workspace_bytes();

@@ -447,17 +447,25 @@ wq_status wq_q4k_quantize(const void* W, int64_t N, int64_t K, void* blocks,
                                          reinterpret_cast<cudaStream_t>(stream), dev.sms));
 }
 
-wq_status wq_q4k_matmul(const void* X, int64_t M, const void* blocks, int64_t N, int64_t K,
-                        void* Y, int out_dtype, wq_stream_t stream) {
+wq_status wq_q4k_matmul_ex(const void* X, int64_t M, const void* blocks, int64_t N,
+                           int64_t K, void* Y, int out_dtype, unsigned int flags,
+                           wq_stream_t stream) {
   if (wq_q4k_bytes(N, K) == 0 || M < 1 || M > 8 || !X || !blocks || !Y)
     return WQ_ERR_INVALID_ARG;
   if (out_dtype != WQ_OUT_F32 && out_dtype != WQ_OUT_BF16) return WQ_ERR_INVALID_ARG;
+  if ((flags & ~unsigned(WQ_MATMUL_STATIC_WEIGHTS)) != 0) return WQ_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(blocks) || !aligned16(Y)) return WQ_ERR_ALIGNMENT;
   DeviceInfo dev;
   if (!wqh::device_info(&dev)) return WQ_ERR_CUDA;
   return from_cuda(wqh::run_q4k_matmul(X, int(M), blocks, int(N), int(K), Y,
                                        out_dtype == WQ_OUT_BF16,
+                                       (flags & WQ_MATMUL_STATIC_WEIGHTS) != 0,
                                        reinterpret_cast<cudaStream_t>(stream), dev.sms));
+}
+
+wq_status wq_q4k_matmul(const void* X, int64_t M, const void* blocks, int64_t N, int64_t K,
+                        void* Y, int out_dtype, wq_stream_t stream) {
+  return wq_q4k_matmul_ex(X, M, blocks, N, K, Y, out_dtype, 0u, stream);
 }
 
 }  // extern "C"
