@@ -57,12 +57,6 @@ struct Params {
   uint32_t off_ring;       // [16 warps][DEPTH][2,304 bytes]
 };
 
-__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
-  return v;
-}
-
 // small non-negative integer (< 2^22) -> binary32, exactly
 __device__ __forceinline__ float small_u2f(uint32_t v) {
   return __uint_as_float(0x4B000000u | v) - 8388608.f;
