@@ -2,8 +2,9 @@
 dequantized weights in tensor memory (gemm2.cuh): shared-memory rings in
 bounds and 1024-byte aligned (the 128-byte swizzle of the activation boxes
 and the 64/128-byte swizzle of the code boxes), copy boxes inside the TMA
-limits with 16-byte aligned inner extents, the tile count and persistent
-grid, and the kernel's scope (groups 32/64/128, K a multiple of 128: a load
+limits with 16-byte aligned inner extents, the epilogue's output staging
+(8 warps x two 2 KB buffers, 1024-byte aligned, after the rings, where it
+fits), the tile count and persistent grid, and the kernel's scope (groups 32/64/128, K a multiple of 128: a load
 stage is 128 k, eight MMAs of K = 16)."""
 import ctypes
 import os
@@ -13,7 +14,7 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 LIB = os.path.join(ROOT, "w4a16_decode_matmul_b200", "libwq.so")
 FIELDS = ["M", "N", "K", "ngroups", "tiles_t", "tiles_w", "num_tiles", "codes_stage_bytes",
-          "smem", "grid"]
+          "smem", "grid", "off_out"]
 SMEM_OPTIN, SMS = 232448, 148
 BW = 128
 BK, HEAD = 128, 1024
@@ -68,7 +69,16 @@ def test_plan_gemm2(lib, M, N, K, bits, group):
     # tensors) when K / group is a multiple of 8 (the tensor maps' row pitch)
     meta = 8 * 2 * 128 * 8 * 2 if (K // group) % 8 == 0 else 0
     assert (off_codes + STAGES * p["codes_stage_bytes"]) % 128 == 0
-    assert p["smem"] == off_codes + STAGES * p["codes_stage_bytes"] + meta <= SMEM_OPTIN
+    rings = off_codes + STAGES * p["codes_stage_bytes"] + meta
+    staging = 8 * 2 * 16 * 32 * 4
+    off_out = -(-rings // 1024) * 1024
+    if off_out + staging <= SMEM_OPTIN:
+        assert p["off_out"] == off_out and p["smem"] == off_out + staging
+    else:
+        assert p["off_out"] == 0 and p["smem"] == rings
+    assert p["smem"] <= SMEM_OPTIN
+    # 4-bit codes always leave room for the staging
+    assert bits == 8 or p["off_out"] != 0
     # every TMA x coordinate (k * 2 bytes for X: stage start and start + 64;
     # bytes for the codes) stays a multiple of 16 bytes
     assert (BK * 2) % 16 == 0 and (64 * 2) % 16 == 0 and row % 16 == 0

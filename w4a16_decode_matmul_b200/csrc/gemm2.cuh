@@ -40,8 +40,12 @@
 //               (A stage s sits beside load stage s: both are freed by the
 //               one commit of the stage's MMAs);
 //   warps 6-13  epilogue: one row of W and 64 tokens per thread; per group
-//               S += s_g D_g in registers; S is written to Y at the end of
-//               the tile.
+//               S += s_g D_g in registers (the row's eight scales of a
+//               block in one 16-byte load); at the end of the tile S goes
+//               out through shared memory by tensor stores, 16 tokens at a
+//               time in two buffers per warp, so that the warps are free for
+//               the next tile's groups while it is written (plain stores
+//               where Y's pitch or shared memory does not allow it).
 // Every wait is bounded in time; a timeout records WQ_ERR_TIMEOUT, sets the
 // CTA's abort flag, the roles stop, issued copies and MMAs are drained and
 // tensor memory is freed.
@@ -99,6 +103,13 @@ constexpr int kBarMetaFull = 38;               // [kMetaSlots] block landed (tx)
 constexpr int kBarMetaEmpty = 46;              // [kMetaSlots] block read by every user
 constexpr int kMetaTensorBytes = kBW * kMetaGroups * 2;  // 2 KB: 128 rows x 8 binary16
 constexpr int kMetaSlotBytes = 2 * kMetaTensorBytes;     // scales, then zeros
+// Output staging: each epilogue warp writes its 32 rows x 16 tokens of Y
+// into one of two buffers and one lane copies it out with a tensor store,
+// so the tile's results leave while the warp starts on the next tile.
+constexpr int kOutChunk = 16;                          // tokens per store
+constexpr int kOutBufBytes = kOutChunk * 32 * 4;       // 2 KB (binary32; bfloat16 uses half)
+constexpr int kOutWarpBytes = 2 * kOutBufBytes;
+__host__ __device__ constexpr int out_stage_bytes(int ew) { return ew * kOutWarpBytes; }
 constexpr int kTmemSlot = 512;                 // byte offset of the TMEM base address
 constexpr int kAbortSlot = 516;                // byte offset of the abort flag
 constexpr int kSmemHead = 1024;
@@ -113,6 +124,7 @@ struct Params {
   uint32_t codes_stage_bytes;  // kBW * kBK * bits / 8
   uint32_t off_x, off_codes;   // rings (1024-byte aligned)
   uint32_t off_meta;           // ring of scale / zero blocks (with MT)
+  uint32_t off_out;            // output staging buffers; 0: plain stores
 };
 
 // A in tensor memory (M = 128 lanes, K = 16 as eight 32-bit columns of
@@ -220,7 +232,8 @@ __global__ void __launch_bounds__(threads_for(DW, EW), 1)
     gemm2_kernel(const __grid_constant__ CUtensorMap tm_x,
                  const __grid_constant__ CUtensorMap tm_codes,
                  const __grid_constant__ CUtensorMap tm_scales,
-                 const __grid_constant__ CUtensorMap tm_zeros, const Params p) {
+                 const __grid_constant__ CUtensorMap tm_zeros,
+                 const __grid_constant__ CUtensorMap tm_y, const Params p) {
   static_assert(G == 32 || G == 64 || G == 128, "group");
   static_assert(LS >= 2 && LS <= kMaxLoadStages && (DW == 4 || DW == 8) &&
                     (EW == 8 || EW == 16), "roles");
@@ -525,81 +538,114 @@ __global__ void __launch_bounds__(threads_for(DW, EW), 1)
     const int half = e >> 2;              // tokens kEpiCols * half .. of the tile
     const int r = 32 * quarter + lane;    // row of the W tile
     const uint32_t lanes = uint32_t(32 * quarter) << 16;
-    int gcount = 0, mb = 0;
+    const bool staged = p.off_out != 0;
+    const bool out_bf16 = p.Y_f32 == nullptr;
+    const uint32_t out0 = smem_addr(smem + p.off_out) + uint32_t(e * kOutWarpBytes);
+    int gcount = 0, mb = 0, chunks = 0;
     bool stop = false;
+    float S[kEpiCols];
+    // S += sg * D_g for the next group's accumulator, read in loads of up to
+    // 32 columns; the buffer is handed back once its last load has landed
+    // in registers, before the last multiply-adds.  False if a wait gave up.
+    auto group = [&](float sg) -> bool {
+      const int db = gcount & 1;
+      if (!wait(kBarDFull + db, uint32_t(gcount >> 1) & 1u)) return false;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + lanes + uint32_t(db * kDCols + half * kEpiCols);
+      constexpr int kLd = kEpiCols < 32 ? kEpiCols : 32;
+#pragma unroll
+      for (int h = 0; h < kEpiCols / kLd; ++h) {
+        float dv[kLd];
+        if constexpr (kLd == 32)
+          tmem_ld32(taddr + uint32_t(32 * h), dv);
+        else
+          tmem_ld16(taddr + uint32_t(16 * h), dv);
+        tmem_wait_ld();
+        if (h == kEpiCols / kLd - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars[kBarDEmpty + db]);
+        }
+#pragma unroll
+        for (int j = 0; j < kLd; ++j) S[kLd * h + j] = fmaf(sg, dv[j], S[kLd * h + j]);
+      }
+      ++gcount;
+      return true;
+    };
     for (int tile = blockIdx.x; tile < p.num_tiles && !stop; tile += gridDim.x) {
       const int t0 = (tile / p.tiles_w) * kBT, w0 = (tile % p.tiles_w) * kBW;
       const int row = w0 + r;
       const bool row_ok = row < p.N;
-      const __half* srow = p.scales + size_t(row_ok ? row : 0) * p.ngroups;
-      float S[kEpiCols];
 #pragma unroll
       for (int j = 0; j < kEpiCols; ++j) S[j] = 0.f;
-      int done = 0;
-      for (int gi = 0; gi < p.ngroups; ++gi, ++gcount) {
-        float sg;
-        if constexpr (MT) {
+      if constexpr (MT) {
+        // the row's eight scales of a block in one 16-byte load; the block
+        // is released as soon as they are in registers
+        for (int gb = 0; gb < p.ngroups && !stop; gb += kMetaGroups) {
           const int ms = mb % kMetaSlots;
-          if (gi % kMetaGroups == 0 && !wait(kBarMetaFull + ms, uint32_t(mb / kMetaSlots) & 1u)) {
+          if (!wait(kBarMetaFull + ms, uint32_t(mb / kMetaSlots) & 1u)) {
             stop = true;
             break;
           }
-          sg = __half2float(reinterpret_cast<const __half*>(smem + p.off_meta +
-                                                            ms * kMetaSlotBytes)[r * kMetaGroups +
-                                                                                 gi % kMetaGroups]);
-          if (gi % kMetaGroups == kMetaGroups - 1 || gi == p.ngroups - 1) {
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[kBarMetaEmpty + ms]);
-            ++mb;
-          }
-        } else {
-          sg = row_ok ? __half2float(srow[gi]) : 0.f;
-        }
-        const int db = gcount & 1;
-        if (!wait(kBarDFull + db, uint32_t(gcount >> 1) & 1u)) {
-          stop = true;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t taddr = tmem_base + lanes + uint32_t(db * kDCols + half * kEpiCols);
-        if constexpr (kEpiCols <= 32) {
-          // one load and one wait per group
-          float dv[32];
-          if constexpr (kEpiCols == 32) {
-            tmem_ld32(taddr, dv);
-          } else {
-            float d16[16];
-            tmem_ld16(taddr, d16);
+          const uint4 sv = lds128(smem_addr(smem + p.off_meta + ms * kMetaSlotBytes) +
+                                  uint32_t(r * kMetaGroups * 2));
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars[kBarMetaEmpty + ms]);
+          ++mb;
+          const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
-            for (int j = 0; j < 16; ++j) dv[j] = d16[j];
-          }
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < kEpiCols; ++j) S[j] = fmaf(sg, dv[j], S[j]);
-        } else {
-          float dv[16];
-#pragma unroll
-          for (int h = 0; h < kEpiCols / 16; ++h) {
-            tmem_ld16(taddr + 16 * h, dv);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 16; ++j) S[16 * h + j] = fmaf(sg, dv[j], S[16 * h + j]);
+          for (int u = 0; u < kMetaGroups; ++u) {
+            const uint32_t bits16 = (u & 1) ? (sw[u >> 1] >> 16) : (sw[u >> 1] & 0xFFFFu);
+            if (!group(__half2float(__ushort_as_half(static_cast<unsigned short>(bits16))))) {
+              stop = true;
+              break;
+            }
           }
         }
-        // D_g is read: the MMA warp may overwrite this buffer
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[kBarDEmpty + db]);
-        done = gi + 1;
+      } else {
+        const __half* srow = p.scales + size_t(row_ok ? row : 0) * p.ngroups;
+        for (int gi = 0; gi < p.ngroups; ++gi) {
+          if (!group(row_ok ? __half2float(srow[gi]) : 0.f)) {
+            stop = true;
+            break;
+          }
+        }
       }
-      if (stop || done != p.ngroups || *abort_flag) break;
-      if (row_ok) {
-        const int tb = t0 + half * kEpiCols;
+      if (stop || *abort_flag) break;
+      const int tb = t0 + half * kEpiCols;
+      if (staged) {
+        // chunk c of 16 tokens into buffer (chunks & 1), once the store that
+        // last read that buffer (two chunks ago) has read it; the tensor
+        // store leaves out the rows past N and the tokens past M
+#pragma unroll
+        for (int c = 0; c < kEpiCols / kOutChunk; ++c, ++chunks) {
+          const uint32_t buf = out0 + uint32_t(chunks & 1) * kOutBufBytes;
+          if (lane == 0) bulk_wait_group_read<1>();
+          __syncwarp();
+          if (out_bf16) {
+#pragma unroll
+            for (int j = 0; j < kOutChunk; ++j)
+              sts16(buf + uint32_t(j * 64 + lane * 2),
+                    __bfloat16_as_ushort(__float2bfloat16_rn(S[kOutChunk * c + j])));
+          } else {
+#pragma unroll
+            for (int j = 0; j < kOutChunk; ++j)
+              sts32(buf + uint32_t(j * 128 + lane * 4), S[kOutChunk * c + j]);
+          }
+          fence_async_shared();
+          __syncwarp();
+          if (lane == 0) {
+            if (tb + kOutChunk * c < p.M && w0 + 32 * quarter < p.N)
+              tma_store_2d(&tm_y, buf, w0 + 32 * quarter, tb + kOutChunk * c);
+            bulk_commit_group();
+          }
+        }
+      } else if (row_ok) {
 #pragma unroll
         for (int j = 0; j < kEpiCols; ++j) {
           const int m = tb + j;
           if (m < p.M) {
-            if (p.Y_f32 != nullptr)
+            if (!out_bf16)
               p.Y_f32[size_t(m) * p.N + row] = S[j];
             else
               p.Y_bf16[size_t(m) * p.N + row] = __float2bfloat16_rn(S[j]);
@@ -607,6 +653,8 @@ __global__ void __launch_bounds__(threads_for(DW, EW), 1)
         }
       }
     }
+    // every tensor store has finished before the CTA's shared memory goes
+    if (staged && lane == 0) bulk_wait_group<0>();
   }
 
   // tensor memory is freed by the warp that allocated it, after every reader

@@ -12,6 +12,7 @@ struct Gemm2Plan {
   wq::gemm2::Params p;
   int grid = 1;
   size_t smem = 0;
+  size_t smem_rings = 0;  // without the output staging
   int variant = 0;
   int bt = 128;   // tokens per tile: 64 for M <= 64 (the MMA's N), else 128
   bool meta_tma = false;  // scales / zeros by TMA (K / group a multiple of 8)
@@ -58,6 +59,15 @@ bool plan_gemm2(int M, int N, int K, int bits, int group, const DeviceInfo& dev,
   plan->meta_tma = p.ngroups % kMetaGroups == 0;
   plan->smem = p.off_meta + (plan->meta_tma ? size_t(kMetaSlots) * kMetaSlotBytes : 0);
   if (plan->smem > size_t(dev.max_smem_optin)) return false;
+  plan->smem_rings = plan->smem;
+  // the epilogue's output staging after the rings, where it fits (not with
+  // 8-bit codes and 128-token tiles)
+  const int ew = M <= 64 ? 8 : kGemm2Variants[variant].epilogue_warps;
+  const size_t off_out = (plan->smem + 1023) & ~size_t(1023);
+  if (off_out + size_t(out_stage_bytes(ew)) <= size_t(dev.max_smem_optin)) {
+    p.off_out = uint32_t(off_out);
+    plan->smem = off_out + size_t(out_stage_bytes(ew));
+  }
   plan->grid = std::min(p.num_tiles, dev.sms);
   return true;
 }
@@ -100,7 +110,25 @@ cudaError_t launch_gemm2(Gemm2Plan* plan, const DeviceInfo* dev, const void* X, 
                            uint64_t(p.N), uint32_t(kMetaGroups), uint32_t(kBW)))
       return cudaErrorInvalidValue;
   }
-  kernel<<<plan->grid, threads_for(DW, EW), plan->smem, s>>>(tx, tc, ts, tz, p);
+  // Y [M][N] for the epilogue's tensor stores: boxes of 32 rows of W x 16
+  // tokens; without the staging (or a map) the epilogue stores directly
+  CUtensorMap ty;
+  std::memcpy(&ty, &tx, sizeof(tx));
+  wq::gemm2::Params pl = p;
+  size_t smem = plan->smem;
+  if (pl.off_out != 0) {
+    const bool f32 = pl.Y_f32 != nullptr;
+    const void* y = f32 ? static_cast<const void*>(pl.Y_f32) : static_cast<const void*>(pl.Y_bf16);
+    const int esz = f32 ? 4 : 2;
+    if (reinterpret_cast<uintptr_t>(y) % 16 != 0 || (int64_t(p.N) * esz) % 16 != 0 ||
+        !encode_2d(&ty, y, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                   esz, uint64_t(p.N), uint64_t(p.M), 32u, uint32_t(kOutChunk))) {
+      pl.off_out = 0;
+      smem = plan->smem_rings;
+      std::memcpy(&ty, &tx, sizeof(tx));
+    }
+  }
+  kernel<<<plan->grid, threads_for(DW, EW), smem, s>>>(tx, tc, ts, tz, ty, pl);
   return cudaGetLastError();
 }
 
@@ -146,8 +174,8 @@ bool run_gemm2(const MatmulArgs& a, cudaError_t* err) {
 extern "C" {
 
 // Test hook, not part of the public ABI: the prefill plan with the weights in
-// tensor memory, written to out[0..9] (M, N, K, ngroups, tiles_t, tiles_w,
-// num_tiles, codes_stage_bytes, smem, grid).  Returns 0 if the shape is
+// tensor memory, written to out[0..10] (M, N, K, ngroups, tiles_t, tiles_w,
+// num_tiles, codes_stage_bytes, smem, grid, off_out).  Returns 0 if the shape is
 // outside the kernel's scope.
 int wq_internal_plan_gemm2(int M, int N, int K, int bits, int group, int sms, int smem_optin,
                            int64_t* out) {
@@ -159,7 +187,7 @@ int wq_internal_plan_gemm2(int M, int N, int K, int bits, int group, int sms, in
   const wq::gemm2::Params& p = plan.p;
   const int64_t v[] = {p.M,         p.N,         p.K,         p.ngroups,         p.tiles_t,
                        p.tiles_w,   p.num_tiles, p.codes_stage_bytes, int64_t(plan.smem),
-                       plan.grid};
+                       plan.grid,   p.off_out};
   for (size_t i = 0; i < sizeof(v) / sizeof(v[0]); ++i) out[i] = v[i];
   return 1;
 }
