@@ -18,12 +18,15 @@ struct Gemm2Plan {
   bool meta_tma = false;  // scales / zeros by TMA (K / group a multiple of 8)
 };
 
-// Build variants (load stages, dequantize warps), chosen through an internal
-// tuning hook.
+// Build variants (load stages, dequantize warps, epilogue warps), chosen
+// through an internal tuning hook.  Eight dequantize warps (two per lane
+// quarter, half of a stage's k each) measured slower on B200 (658 against
+// 757 TFLOP/s at M = 2048: at 576 threads the registers run out and the
+// epilogue spills), so one build remains.
 struct Gemm2Variant {
   int load_stages, dequant_warps, epilogue_warps;
 };
-constexpr Gemm2Variant kGemm2Variants[] = {{4, 4, 8}, {4, 8, 8}};
+constexpr Gemm2Variant kGemm2Variants[] = {{4, 4, 8}};
 constexpr int kNumGemm2Variants = int(sizeof(kGemm2Variants) / sizeof(kGemm2Variants[0]));
 int g_gemm2_variant = 0;
 
@@ -136,10 +139,7 @@ template <int BITS, bool SYM, int G, bool MT>
 cudaError_t launch_gemm2_v(Gemm2Plan* plan, const DeviceInfo* dev, const void* X, const void* c,
                            const void* sc, const void* z, cudaStream_t s) {
   if (plan->bt == 64) return launch_gemm2<BITS, SYM, G, 6, 4, 8, 64, MT>(plan, dev, X, c, sc, z, s);
-  switch (plan->variant) {
-    case 1: return launch_gemm2<BITS, SYM, G, 4, 8, 8, 128, MT>(plan, dev, X, c, sc, z, s);
-    default: return launch_gemm2<BITS, SYM, G, 4, 4, 8, 128, MT>(plan, dev, X, c, sc, z, s);
-  }
+  return launch_gemm2<BITS, SYM, G, 4, 4, 8, 128, MT>(plan, dev, X, c, sc, z, s);
 }
 
 template <int BITS, bool SYM, int G>
@@ -193,8 +193,8 @@ int wq_internal_plan_gemm2(int M, int N, int K, int bits, int group, int sms, in
 }
 
 // Tuning hook, not part of the public ABI: the build variant of the prefill
-// kernel with the weights in tensor memory (0 .. 1, see kGemm2Variants; one
-// that does not fit falls back to 0).  Returns the number of variants.
+// kernel with the weights in tensor memory (see kGemm2Variants; one that
+// does not fit falls back to 0).  Returns the number of variants.
 int wq_internal_set_gemm2_variant(int variant) {
   if (variant >= 0 && variant < wqh::kNumGemm2Variants) wqh::g_gemm2_variant = variant;
   return wqh::kNumGemm2Variants;
