@@ -50,9 +50,12 @@ bool plan_ks(int M, int N, int K, int bits, int group, const DeviceInfo& dev, Ks
 
 template <bool SYM, int MT, int DEPTH>
 cudaError_t launch_ks(KsPlan* plan, const DeviceInfo& dev, cudaStream_t s, bool pdl) {
-  auto kernel = &wq::ks::gemv_ks_kernel<SYM, MT, DEPTH>;
-  static int configured[kMaxDevices] = {};
-  cudaError_t e = configure_smem(kernel, configured, size_t(dev.max_smem_optin));
+  // the build without the bounds-checked refill where every tile is whole
+  auto kernel = plan->p.N % wq::ks::kTileRows == 0 ? &wq::ks::gemv_ks_kernel<SYM, MT, DEPTH, false>
+                                                   : &wq::ks::gemv_ks_kernel<SYM, MT, DEPTH, true>;
+  static int configured[2][kMaxDevices] = {};  // per build
+  cudaError_t e = configure_smem(kernel, configured[plan->p.N % wq::ks::kTileRows == 0 ? 0 : 1],
+                                 size_t(dev.max_smem_optin));
   if (e != cudaSuccess) return e;
   plan->p.pdl = pdl ? 1 : 0;
   cudaLaunchConfig_t cfg = {};
