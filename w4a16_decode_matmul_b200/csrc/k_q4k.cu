@@ -56,9 +56,12 @@ bool plan_q4ks(int M, int N, int K, const DeviceInfo& dev, Q4ksPlan* plan) {
 
 template <int DEPTH>
 cudaError_t launch_q4ks(Q4ksPlan* plan, const DeviceInfo& dev, cudaStream_t s) {
-  auto kernel = &wq::q4ks::gemv_q4k_kernel<DEPTH>;
-  static int configured[kMaxDevices] = {};
-  const cudaError_t e = configure_smem(kernel, configured, size_t(dev.max_smem_optin));
+  // the build without the bounds-checked copies where every tile is whole
+  const bool whole = plan->p.N % wq::q4ks::kTileRows == 0;
+  auto kernel = whole ? &wq::q4ks::gemv_q4k_kernel<DEPTH, false>
+                      : &wq::q4ks::gemv_q4k_kernel<DEPTH, true>;
+  static int configured[2][kMaxDevices] = {};  // per build
+  const cudaError_t e = configure_smem(kernel, configured[whole ? 0 : 1], size_t(dev.max_smem_optin));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attrs[1];

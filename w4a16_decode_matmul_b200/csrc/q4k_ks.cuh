@@ -62,7 +62,9 @@ __device__ __forceinline__ float small_u2f(uint32_t v) {
   return __uint_as_float(0x4B000000u | v) - 8388608.f;
 }
 
-template <int DEPTH>
+// RAGGED: N is not a multiple of 16, so the last tile holds rows past N
+// (their copies are zero-filled); without it every copy is unconditional.
+template <int DEPTH, bool RAGGED = true>
 __global__ void __launch_bounds__(kThreads, 2) gemv_q4k_kernel(const Params p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -90,7 +92,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_q4k_kernel(const Params p) {
 #pragma unroll
       for (int i = 0; i < 6; ++i) {
         if (crow + 3 * i < kTileRows) {
-          const bool ok = fetched < nfull || row0 + 3 * i < p.N;
+          const bool ok = !RAGGED || fetched < nfull || row0 + 3 * i < p.N;
           ld::cp_async16(dst + 3 * kBlockBytes * i, ok ? tbase + size_t(3 * i) * kRowBytes : p.blocks,
                          ok);
         }
