@@ -3,8 +3,9 @@ same seeded inputs against the oracle: the balanced kernel with and without
 its workspace (row tiles summed across CTAs, or whole tiles per SM), under
 programmatic dependent launch, the cluster-split kernel it replaces for
 M <= 8, the direct-load kernel (4-bit codes, groups of 128, M <= 4), the
-bulk-staged kernel (the same formats, K a multiple of 1,024) and the
-k-sliced direct-load kernel (the same formats, K = 4096).  Tolerance as in test_matmul_gpu: |y - y_ref| <= 1e-4 sum|x w|
+bulk-staged kernel (the same formats, K a multiple of 1,024), the
+k-sliced direct-load kernel (the same formats, K = 4096) and the
+tensor-memory kernel (4- and 8-bit codes, groups of 128, K = 4096, M <= 2).  Tolerance as in test_matmul_gpu: |y - y_ref| <= 1e-4 sum|x w|
 (+ one bfloat16 ulp for bfloat16 out)."""
 import contextlib
 import ctypes
@@ -19,7 +20,7 @@ from tests.gpu_util import check_tolerance, host_bits, oracle_quantize, weight, 
 
 pytestmark = pytest.mark.gpu
 
-AUTO, CLUSTER, BALANCED, BALANCED_SPLIT, DIRECT, BULK, KSLICE = 0, 1, 2, 3, 4, 5, 6
+AUTO, CLUSTER, BALANCED, BALANCED_SPLIT, DIRECT, BULK, KSLICE, TMEM = 0, 1, 2, 3, 4, 5, 6, 7
 
 
 @contextlib.contextmanager
@@ -50,8 +51,9 @@ def workspace_clear():
 
 SHAPES = [(1, 14336, 4096), (2, 1000, 4096), (3, 4096, 4096), (5, 1024, 4096), (8, 700, 4096),
           (1, 4096, 14336), (2, 520, 14336), (1, 77, 1024), (4, 300, 2048), (1, 1201, 8192),
-          (4, 1203, 4096), (1, 5, 4096)]
-FORMATS = [(4, 128, False), (4, 128, True), (4, 64, True), (4, 32, False), (8, 128, False), (8, 64, True),
+          (4, 1203, 4096), (1, 5, 4096), (2, 1203, 4096)]
+FORMATS = [(4, 128, False), (4, 128, True), (4, 64, True), (4, 32, False), (8, 128, False),
+           (8, 128, True), (8, 64, True),
            (8, 32, False)]
 
 
@@ -105,6 +107,12 @@ def test_balanced_kernel_modes(M, N, K, bits, group, sym):
             outs["kslice"] = wq().matmul(Xd, qw)
             outs["kslice_pdl"] = wq().matmul(Xd, qw, static_weights=True)
             outs["kslice_bf16"] = wq().matmul(Xd, qw, out_dtype=torch.bfloat16)
+    tmem = group == 128 and M <= 2 and K == 4096
+    if tmem:
+        with kernel(TMEM):
+            outs["tmem"] = wq().matmul(Xd, qw)
+            outs["tmem_pdl"] = wq().matmul(Xd, qw, static_weights=True)
+            outs["tmem_bf16"] = wq().matmul(Xd, qw, out_dtype=torch.bfloat16)
     outs["auto"] = wq().matmul(Xd, qw, static_weights=True)
     torch.cuda.synchronize()
     assert wq().get_device_error() == 0
@@ -121,9 +129,11 @@ def test_balanced_kernel_modes(M, N, K, bits, group, sym):
         assert torch.equal(outs["bulk"], outs["bulk_pdl"])
     if kslice:
         assert torch.equal(outs["kslice"], outs["kslice_pdl"])
+    if tmem:
+        assert torch.equal(outs["tmem"], outs["tmem_pdl"])
 
 
-@pytest.mark.parametrize("choice", [AUTO, BULK, KSLICE])
+@pytest.mark.parametrize("choice", [AUTO, BULK, KSLICE, TMEM])
 def test_back_to_back_static_weights(choice):
     """A chain of launches with programmatic dependent launch, each over a
     different copy of the weights and reading the previous call's output as
@@ -150,7 +160,7 @@ def test_back_to_back_static_weights(choice):
     assert workspace_clear()
 
 
-@pytest.mark.parametrize("choice", [AUTO, BULK, KSLICE])
+@pytest.mark.parametrize("choice", [AUTO, BULK, KSLICE, TMEM])
 def test_graph_replay_with_static_weights(choice):
     """Captured in a CUDA graph (the bench's launch mode), replayed twice."""
     N, K = 14336, 4096
@@ -175,7 +185,7 @@ def test_graph_replay_with_static_weights(choice):
     assert wq().get_device_error() == 0
 
 
-@pytest.mark.parametrize("bits,group,sym", [(4, 128, False), (8, 32, True)])
+@pytest.mark.parametrize("bits,group,sym", [(4, 128, False), (8, 32, True), (8, 128, False)])
 def test_activation_rows_of_wide_dynamic_range(bits, group, sym):
     """The balanced kernel rounds each activation row to binary16 after a
     power-of-two scaling that puts the row's largest magnitude near 2^15:
@@ -202,3 +212,9 @@ def test_activation_rows_of_wide_dynamic_range(bits, group, sym):
                 Y = wq().matmul(X.cuda(), qw)
             torch.cuda.synchronize()
             check_tolerance(Y.cpu().numpy(), y_ref, y_abs, False)
+    if group == 128:
+        with kernel(TMEM):  # two rows at a time: the kernel's scope is M <= 2
+            for m0 in (0, 2):
+                Y = wq().matmul(X[m0:m0 + 2].cuda(), qw)
+                torch.cuda.synchronize()
+                check_tolerance(Y.cpu().numpy(), y_ref[m0:m0 + 2], y_abs[m0:m0 + 2], False)

@@ -77,6 +77,7 @@ struct MatmulArgs {
 bool run_ld(const MatmulArgs& a, cudaError_t* err);
 bool run_tb(const MatmulArgs& a, cudaError_t* err);
 bool run_ks(const MatmulArgs& a, cudaError_t* err);
+bool run_tc(const MatmulArgs& a, cudaError_t* err);
 bool run_sk(const MatmulArgs& a, bool split, cudaError_t* err);
 bool run_gemv(const MatmulArgs& a, cudaError_t* err);
 bool run_gemm(const MatmulArgs& a, cudaError_t* err);

@@ -235,6 +235,10 @@ wq_status wq_matmul(const void* X, int64_t M, const void* codes, const void* sca
     if (wqh::run_ks(a, &e)) return from_cuda(e);
     return WQ_ERR_UNSUPPORTED;
   }
+  if (choice == 7) {
+    if (wqh::run_tc(a, &e)) return from_cuda(e);
+    return WQ_ERR_UNSUPPORTED;
+  }
   if (choice == 4 || choice == 0) {
     if (wqh::run_ld(a, &e)) return from_cuda(e);
     if (choice == 4) return WQ_ERR_UNSUPPORTED;
@@ -360,7 +364,8 @@ const char* wq_internal_last_cuda_error(void) { return cudaGetErrorName(g_last_c
 // the small-batch kernel, 1 forces the cluster-split kernel, 2 forces the
 // balanced kernel, 3 forces the balanced kernel with row tiles split across
 // CTAs whenever a workspace is given, 4 forces the direct-load kernel, 5 the
-// bulk-staged kernel, 6 the k-sliced direct-load kernel (2 to 6 return
+// bulk-staged kernel, 6 the k-sliced direct-load kernel, 7 the tensor-memory
+// small-batch kernel (2 to 7 return
 // WQ_ERR_UNSUPPORTED where the forced kernel does not apply).
 void wq_internal_set_kernel(int choice) { wqh::g_kernel_choice = choice; }
 
