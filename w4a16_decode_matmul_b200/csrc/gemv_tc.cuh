@@ -128,6 +128,59 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
   for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Four 8-bit codes -> (u0, u1), (u2, u3) as exact bfloat16 pairs: binary32
+// 2^23 + u by byte permutes, minus 2^23 two at a time (exact), then one
+// packing conversion per pair (exact: u < 256).
+__device__ __forceinline__ void unpack_u8_pairs(uint32_t w, uint32_t (&r)[2]) {
+  asm("{\n\t"
+      ".reg .b32 f0, f1, f2, f3;\n\t"
+      ".reg .b64 p, q;\n\t"
+      "prmt.b32 f0, %2, %3, 0x7650;\n\t"
+      "prmt.b32 f1, %2, %3, 0x7651;\n\t"
+      "prmt.b32 f2, %2, %3, 0x7652;\n\t"
+      "prmt.b32 f3, %2, %3, 0x7653;\n\t"
+      "mov.b64 p, {f0, f1};\n\t"
+      "mov.b64 q, {f2, f3};\n\t"
+      "sub.rn.f32x2 p, p, %4;\n\t"
+      "sub.rn.f32x2 q, q, %4;\n\t"
+      "mov.b64 {f0, f1}, p;\n\t"
+      "mov.b64 {f2, f3}, q;\n\t"
+      "cvt.rn.bf16x2.f32 %0, f1, f0;\n\t"
+      "cvt.rn.bf16x2.f32 %1, f3, f2;\n\t"
+      "}"
+      : "=r"(r[0]), "=r"(r[1])
+      : "r"(w), "r"(0x4B000000u), "l"(0x4B0000004B000000ull));
+}
+
+// The eight MMAs of one half and tile (M = 128, N from idesc, K = 16 each):
+// A columns a, a + 8, ..., a + 56 in tensor memory, B descriptors bd[k];
+// the first overwrites the accumulator d, the rest add to it.
+__device__ __forceinline__ void mma8(uint32_t d, uint32_t a, const uint64_t (&bd)[8],
+                                     uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b32 ak;\n\t"
+      "setp.ne.b32 p, %11, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %10, p;\n\t"
+      "setp.eq.b32 p, %11, 0;\n\t"
+      "add.u32 ak, %1, 8;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], %3, %10, p;\n\t"
+      "add.u32 ak, %1, 16;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], %4, %10, p;\n\t"
+      "add.u32 ak, %1, 24;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], %5, %10, p;\n\t"
+      "add.u32 ak, %1, 32;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], %6, %10, p;\n\t"
+      "add.u32 ak, %1, 40;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], %7, %10, p;\n\t"
+      "add.u32 ak, %1, 48;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], %8, %10, p;\n\t"
+      "add.u32 ak, %1, 56;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ak], %9, %10, p;\n\t}" ::"r"(d),
+      "r"(a), "l"(bd[0]), "l"(bd[1]), "l"(bd[2]), "l"(bd[3]), "l"(bd[4]), "l"(bd[5]),
+      "l"(bd[6]), "l"(bd[7]), "r"(idesc), "r"(0u)
+      : "memory");
+}
+
 // Four 16-byte copies: dst[g] + off <- src + STRIDE g.
 template <int STRIDE>
 __device__ __forceinline__ void copy4(const uint32_t (&dst)[4], uint32_t off, const uint8_t* src) {
@@ -298,11 +351,13 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const Params p) {
   const uint32_t tmem_base = *tmem_slot;
 
   // Waits poll with test_wait, reading the time limit and the abort flag
-  // every 64 polls.
-  auto wait = [&](int bar, uint32_t parity) {
+  // every 64 polls; the dequantize warps (idle) sleep briefly between polls
+  // so as to leave issue slots to the MMA thread of their sub-partition.
+  auto wait = [&](int bar, uint32_t parity, bool idle) {
     if (mbar_test_wait(&bars[bar], parity)) return true;
     const unsigned long long start = global_timer_ns();
     for (uint32_t n = 1;; ++n) {
+      if (idle) __nanosleep(32);
       if (mbar_test_wait(&bars[bar], parity)) return true;
       if ((n & 63u) == 0) {
         if (*abort_flag) return false;
@@ -318,26 +373,28 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const Params p) {
   if (warp == kMmaWarp) {
     // ---------------------------------------------------------- MMA issue
     if (lane == 0) {
-      const uint32_t b0 = smem_addr(smem + p.off_b);
+      // B never changes: both halves' eight descriptors, once (k step k: box
+      // k / 4 of the half, 32 bytes further per step in it)
+      uint64_t bd[2][8];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint64_t base = gemm2::umma_desc_sw128(smem_addr(smem + p.off_b) + uint32_t(2 * h * kBox));
+#pragma unroll
+        for (int k = 0; k < 8; ++k) bd[h][k] = base + uint64_t((k >> 2) * (kBox >> 4) + 2 * (k & 3));
+      }
       bool stop = false;
       for (int e = 0; e < ntiles && !stop; ++e) {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int sl = 2 * h + (e & 1);  // A slot, accumulator and barrier of this tile
           // the half's A is written (and the accumulator's previous use read)
-          if (!wait(kBarAFull + sl, uint32_t(e >> 1) & 1u)) {
+          if (!wait(kBarAFull + sl, uint32_t(e >> 1) & 1u, false)) {
             stop = true;
             break;
           }
           gemm2::tc_fence_after();
-          const uint32_t d = tmem_base + uint32_t(kDCol0 + sl * kN);
-          const uint32_t a = tmem_base + uint32_t(sl * kACols);
-          const uint64_t bd = gemm2::umma_desc_sw128(b0 + uint32_t(2 * h * kBox));
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            gemm2::tc_mma_ts(d, a + uint32_t(8 * k),
-                             bd + uint64_t((k >> 2) * (kBox >> 4) + 2 * (k & 3)), kIdesc,
-                             k > 0 ? 1u : 0u);
+          mma8(tmem_base + uint32_t(kDCol0 + sl * kN), tmem_base + uint32_t(sl * kACols), bd[h],
+               kIdesc);
           gemm2::tc_commit(&bars[kBarDone + sl]);
         }
       }
@@ -400,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const Params p) {
                   for (int t = 0; t < 4; ++t) a[16 * c + 4 * e + t] = u[t];
                 } else {
                   uint32_t u[2];
-                  unpack_u8(w4[e], u);  // (u0, u1), (u2, u3)
+                  unpack_u8_pairs(w4[e], u);  // (u0, u1), (u2, u3)
 #pragma unroll
                   for (int t = 0; t < 2; ++t) a[8 * c + 2 * e + t] = u[t];
                 }
@@ -408,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const Params p) {
             }
             if (hh == 0) {
               // warp-uniform: the tensor-memory stores below are .aligned
-              const bool ok = wait(kBarDone + sl, (uint32_t(it >> 1) & 1u) ^ 1u);
+              const bool ok = wait(kBarDone + sl, (uint32_t(it >> 1) & 1u) ^ 1u, true);
               if (!__all_sync(0xffffffffu, ok)) {
                 stop = true;
                 break;
@@ -428,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const Params p) {
         if (it > 0) {
           // tile it - 1: this lane's group sums -> the row's partial sum
           const int e = it - 1, sl = 2 * j + (e & 1);
-          const bool ok = wait(kBarDone + sl, uint32_t(e >> 1) & 1u);
+          const bool ok = wait(kBarDone + sl, uint32_t(e >> 1) & 1u, true);
           if (!__all_sync(0xffffffffu, ok)) {
             stop = true;
             break;
