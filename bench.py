@@ -775,73 +775,131 @@ def _cudart():
             rt.cudaMemcpyAsync.restype = ctypes.c_int
             rt.cudaStreamSynchronize.argtypes = [ctypes.c_void_p]
             rt.cudaStreamSynchronize.restype = ctypes.c_int
+            rt.cudaEventCreateWithFlags.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_uint]
+            rt.cudaEventCreateWithFlags.restype = ctypes.c_int
+            rt.cudaEventRecord.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+            rt.cudaEventRecord.restype = ctypes.c_int
+            rt.cudaEventSynchronize.argtypes = [ctypes.c_void_p]
+            rt.cudaEventSynchronize.restype = ctypes.c_int
+            rt.cudaEventDestroy.argtypes = [ctypes.c_void_p]
+            rt.cudaEventDestroy.restype = ctypes.c_int
             return rt
     return None
 
 
 def measure_e2e(wq, torch, dev, pool, pool_n, args):
-    """End to end through the C ABI with host buffers: every step copies X
-    from pinned host memory to the device (cudaMemcpyAsync), calls
-    wq_matmul, copies Y back to pinned host memory and waits for it (the
-    host reads Y), all inside the timed region (wall clock, max with the
-    device events)."""
+    """End to end through the C ABI with host buffers, pipelined as a
+    serving loop would run it: every step copies its X from pinned host
+    memory to the device (cudaMemcpyAsync), calls wq_matmul and copies its
+    Y back to pinned host memory; steps alternate between two streams with
+    four buffer slots, and before a slot is reused the host waits for that
+    step's Y and reads it.  Everything is inside the timed region (wall
+    clock, max with the device events); at the end every slot's Y is
+    checked against a device result of the same product."""
     import ctypes
     import synth
     lib = wq.lib
     rt = _cudart()
-    Xh = synth.activation(M, K, seed=1).pin_memory()
-    Yh = torch.empty(M, N, dtype=torch.float32).pin_memory()
-    Xd = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
-    Yd = torch.empty(M, N, dtype=torch.float32, device=dev)
-    stream = torch.cuda.Stream(dev)
-    h = ctypes.c_void_p(stream.cuda_stream)
-    ws = wq.workspace(dev, stream.cuda_stream)
+    depth, nstreams = 4, 2
+    x_host = synth.activation(M, K, seed=1)
+    Xh = [x_host.clone().pin_memory() for _ in range(depth)]
+    Yh = [torch.empty(M, N, dtype=torch.float32).pin_memory() for _ in range(depth)]
+    Xd = [torch.empty(M, K, dtype=torch.bfloat16, device=dev) for _ in range(depth)]
+    Yd = [torch.empty(M, N, dtype=torch.float32, device=dev) for _ in range(depth)]
+    streams = [torch.cuda.Stream(dev) for _ in range(nstreams)]
+    handles = [ctypes.c_void_p(st.cuda_stream) for st in streams]
+    wss = [wq.workspace(dev, st.cuda_stream) for st in streams]
     vp = ctypes.c_void_p
+    # per-slot completion events (raw runtime events when the runtime is at
+    # hand: cheaper per step than torch's) and numpy views of the host Y
+    if rt is not None:
+        events = []
+        for _ in range(depth):
+            ev = vp()
+            if rt.cudaEventCreateWithFlags(ctypes.byref(ev), 2) != 0:  # cudaEventDisableTiming
+                raise RuntimeError("cudaEventCreateWithFlags failed")
+            events.append(ev)
+        record = lambda slot, si: rt.cudaEventRecord(events[slot], handles[si])
+        wait_slot = lambda slot: rt.cudaEventSynchronize(events[slot])
+    else:
+        events = [torch.cuda.Event() for _ in range(depth)]
+        record = lambda slot, si: events[slot].record(streams[si])
+        wait_slot = lambda slot: events[slot].synchronize()
+    y_views = [y.numpy() for y in Yh]
     x_bytes, y_bytes = M * K * 2, M * N * 4
-    calls = []
-    for q in pool:
-        calls.append((vp(Xd.data_ptr()), M, vp(q.codes.data_ptr()), vp(q.scales.data_ptr()),
-                      None if q.zeros is None else vp(q.zeros.data_ptr()), N, K, BITS, GROUP,
-                      int(SYM), vp(Yd.data_ptr()), wq.WQ_OUT_F32, vp(ws.data_ptr()), ws.numel(),
-                      0, h))
+
+    def call(i, slot, si):
+        q = pool[i % pool_n]
+        return (vp(Xd[slot].data_ptr()), M, vp(q.codes.data_ptr()), vp(q.scales.data_ptr()),
+                None if q.zeros is None else vp(q.zeros.data_ptr()), N, K, BITS, GROUP, int(SYM),
+                vp(Yd[slot].data_ptr()), wq.WQ_OUT_F32, vp(wss[si].data_ptr()), wss[si].numel(),
+                0, handles[si])
+
+    calls = [[call(i, i % depth, (i % depth) % nstreams) for i in range(pool_n * depth)]]
+    reads = [0.0]
 
     def step(i):
+        slot = i % depth
+        si = slot % nstreams          # a slot always uses the same stream
+        h, st = handles[si], streams[si]
+        if i >= depth:
+            wait_slot(slot)           # step i - depth's Y is on the host: read it
+            reads[0] += float(y_views[slot][0, 0])
         if rt is not None:
-            rt.cudaMemcpyAsync(vp(Xd.data_ptr()), vp(Xh.data_ptr()), x_bytes, 1, h)
+            rt.cudaMemcpyAsync(vp(Xd[slot].data_ptr()), vp(Xh[slot].data_ptr()), x_bytes, 1, h)
         else:
-            with torch.cuda.stream(stream):
-                Xd.copy_(Xh, non_blocking=True)
-        st = lib.wq_matmul(*calls[i % pool_n])
-        if st != 0:
-            raise wq.WQError(st, "wq_matmul")
+            with torch.cuda.stream(st):
+                Xd[slot].copy_(Xh[slot], non_blocking=True)
+        c = calls[0][i % len(calls[0])]
+        status = lib.wq_matmul(*c)
+        if status != 0:
+            raise wq.WQError(status, "wq_matmul")
         if rt is not None:
-            rt.cudaMemcpyAsync(vp(Yh.data_ptr()), vp(Yd.data_ptr()), y_bytes, 2, h)
-            rt.cudaStreamSynchronize(h)
+            rt.cudaMemcpyAsync(vp(Yh[slot].data_ptr()), vp(Yd[slot].data_ptr()), y_bytes, 2, h)
         else:
-            with torch.cuda.stream(stream):
-                Yh.copy_(Yd, non_blocking=True)
-            stream.synchronize()
+            with torch.cuda.stream(st):
+                Yh[slot].copy_(Yd[slot], non_blocking=True)
+        record(slot, si)
+
+    def drain(last):
+        for i in range(max(0, last - depth), last):
+            wait_slot(i % depth)
+            reads[0] += float(y_views[i % depth][0, 0])
 
     steps = max(200, min(5000, args.steps))
+    steps -= steps % (pool_n * depth)  # whole cycles: every weight copy and slot alike
+    steps = max(steps, pool_n * depth)
     with torch.cuda.device(dev):
-        for i in range(20):
+        for i in range(2 * depth):
             step(i)
+        drain(2 * depth)
+        torch.cuda.synchronize(dev)
         s = torch.cuda.Event(enable_timing=True)
         e = torch.cuda.Event(enable_timing=True)
         t0 = time.perf_counter()
-        s.record(stream)
+        s.record(streams[0])
         for i in range(steps):
             step(i)
-        e.record(stream)
+        drain(steps)
+        for st in streams[1:]:
+            streams[0].wait_stream(st)
+        e.record(streams[0])
         torch.cuda.synchronize(dev)
         wall = time.perf_counter() - t0
+    ref = wq.matmul(x_host.to(dev), pool[0])
+    torch.cuda.synchronize(dev)
+    checked = all(torch.equal(Yh[j], ref.cpu()) for j in range(depth))
+    if rt is not None:
+        for ev in events:
+            rt.cudaEventDestroy(ev)
     ms = reduce_max(max(s.elapsed_time(e), wall * 1e3), dev)
     _, world, _ = dist_env()
     return {"value": round(whole_job_gbs(algorithmic_bytes(), steps, world, ms), 3),
             "unit": "GB/s", "h2d_bytes_per_step": x_bytes, "d2h_bytes_per_step": y_bytes,
-            "steps": steps, "us_per_step": round(ms / steps * 1e3, 3),
+            "steps": steps, "us_per_step": round(ms / steps * 1e3, 3), "results_checked": checked,
             "how": ("C ABI wq_matmul per step between cudaMemcpyAsync of X (pinned host -> "
-                    "device) and of Y (device -> pinned host) and a stream synchronize")}
+                    "device) and of Y (device -> pinned host); 4 buffer slots over 2 streams, "
+                    "the host waits for and reads each step's Y before reusing its slot")}
 
 
 def ncu_case(which: str = "decode"):
